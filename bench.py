@@ -1,0 +1,421 @@
+"""Benchmark of the CSA2 decode layer step on B200: Reindex mode at 1M context (batch 128, a pool of
+2000 blocks x 8 positions, Top-512, 16 heads x 128 + a 128-token window).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One JSON line on rank 0. `value` is whole-job queries/s with inputs resident in HBM, timed with
+CUDA events (max over ranks); `e2e` is the same through the C ABI with the step's inputs copied
+from pinned host memory and its outputs copied back inside the timed region. `roofline` reports the
+dominant kernel (the Reindex indexer) against the measured HBM copy bandwidth. `cpu_baseline` times
+the CPU oracle on a bounded sample. With --gpus N > 1 (torchrun), every rank runs its own batch of
+sequences (data parallel, no collective in the data path: weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "CSA2 decode queries/s at 1M ctx; HBM GB/s as % of 8 TB/s roofline"
+UNIT = "queries/s"
+DEFAULT_WORKLOAD = "reindex_b128_n1m"
+
+
+# ---------------------------------------------------------------------------------------------
+# algorithmic bytes (reads of what the step must read, writes of what it must write; no scratch)
+# ---------------------------------------------------------------------------------------------
+def algorithmic_bytes(wl):
+    """Per query: dict kernel -> bytes. Entry sizes: FP4 main row 128 + 16 B, indexer row 128 + 16 B,
+    window row 256 B (FP8)."""
+    k, win = wl.k, wl.win
+    q, out, iq, idx = 16 * 128 * 2, 16 * 128 * 2, 4 * 64 * 2, k * 4
+    attend = k * 144 + win * 256 + q + idx + out
+    if wl.mode == "reindex":
+        index = wl.pool_blocks * wl.bs * 144 + wl.pool_blocks * 4 + 4 + iq + idx
+        append = 256 * 2 + 256
+    elif wl.mode == "full":
+        index = wl.context * 144 + iq + idx + (wl.pool_blocks * 4 + 4 if wl.pool_blocks else 0)
+        append = 3 * 256 * 2 + 144 * 2 + 256
+    elif wl.mode == "minimal":
+        index = 0
+        append = 256 * 2 + 256
+    else:
+        index = wl.context * 144 + iq + idx  # per query row (upper bound: the last row sees all)
+        append = 3 * 256 * 2 + 144 * 2 + 256
+    return {"append": append, "index": index, "attend": attend}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_hash(name):
+    src = os.path.join(ROOT, "compressed_sparse_attention_append_b200", "csrc", name)
+    with open(src, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel_file, workload):
+    """Per-launch DRAM bytes of a kernel from profiles/traffic.txt, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    h = kernel_source_hash(kernel_file)
+    with open(p) as f:
+        for line in f:
+            parts = line.split("#")[0].split()
+            if len(parts) == 4 and parts[0] == kernel_file and parts[1] == workload and parts[2] == h:
+                return int(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.proc or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9 or not c[1].split()[0].isdigit():
+                    continue
+                sm.append(int(c[1].split()[0]))
+                mx = int(c[2].split()[0])
+                for n, v in zip(names, c[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------------------------
+def oracle_sample(wl_name, budget_s=12.0, max_queries=None):
+    """Times the oracle on whole decode steps of sampled sequences of the workload; returns
+    (queries/s, description, threads)."""
+    import numpy as np
+    import torch
+
+    import oracle
+    import workloads as W
+
+    wl = W.WORKLOADS[wl_name]
+    oracle.build()
+    N = wl.context
+    seqs = [0, 1]
+    built = []
+    for b in seqs:
+        bt = torch.tensor([b])
+        c = oracle.SeqCache(cap=N, swa_cap=128)
+        if wl.mode == "reindex":
+            pool = W.distinct_sorted(wl.seed, "pool", bt, N // wl.bs, wl.pool_blocks)[0].to(torch.int32).numpy()
+            for g0 in range(0, wl.pool_blocks, 250):
+                blk = torch.from_numpy(pool[g0:g0 + 250].astype(np.int64))
+                p = (blk.unsqueeze(1) * wl.bs + torch.arange(wl.bs)).reshape(-1)
+                kv = W.cache_values(wl.seed, "kv", bt, p, 256)[0]
+                ik = W.cache_values(wl.seed, "ik", bt, p, 256)[0]
+                for j in range(blk.numel()):
+                    c.append(int(p[j * wl.bs]), kv=kv[j * wl.bs:(j + 1) * wl.bs], idx_k=ik[j * wl.bs:(j + 1) * wl.bs])
+        elif wl.mode == "full":
+            for a in range(0, N - 1, 8192):
+                p = torch.arange(a, min(N - 1, a + 8192))
+                c.append(a, kv=W.cache_values(wl.seed, "kv", bt, p, 256)[0], idx_k=W.cache_values(wl.seed, "ik", bt, p, 256)[0])
+            pool = None
+        else:
+            pool = None
+        pw = torch.arange(N - wl.win, N - 1)
+        c.append(N - wl.win, swa_kv=W.cache_values(wl.seed, "swa", bt, pw, 256)[0])
+        qp = torch.tensor([N - 1])
+        inp = {
+            "swa": W.cache_values(wl.seed, "swa", bt, qp, 256)[0],
+            "iq": W.cache_values(wl.seed, "iq", bt, qp, 256)[0, 0],
+            "q": W.cache_values(wl.seed, "q", bt, qp, 2048)[0, 0],
+            "kv": W.cache_values(wl.seed, "kv", bt, qp, 256)[0],
+            "ik": W.cache_values(wl.seed, "ik", bt, qp, 256)[0],
+        }
+        if wl.mode == "minimal":
+            inp["idx"] = W.distinct_sorted(wl.seed, "sel", bt, N - 1, wl.k)[0].to(torch.int32).numpy()
+            kvr = W.cache_values(wl.seed, "kv", bt, torch.from_numpy(inp["idx"].astype(np.int64)), 256)[0]
+            for j, pp in enumerate(inp["idx"]):
+                c.append(int(pp), kv=kvr[j:j + 1])
+        built.append((c, pool, inp))
+
+    def step(c, pool, inp):
+        if wl.mode == "reindex":
+            c.append(N - 1, swa_kv=inp["swa"])
+            idx = c.index_topk_reindex(N - 1, inp["iq"], pool, len(pool), k=wl.k)
+        elif wl.mode == "full":
+            c.append(N - 1, kv=inp["kv"], idx_k=inp["ik"], swa_kv=inp["swa"])
+            r = c.index_topk_full(N - 1, inp["iq"], k=wl.k, pool_blocks=wl.pool_blocks)
+            idx = r[0] if wl.pool_blocks else r
+        else:
+            c.append(N - 1, swa_kv=inp["swa"])
+            idx = inp["idx"]
+        return c.sparse_attend(N - 1, inp["q"], idx)
+
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        for c, pool, inp in built:
+            step(c, pool, inp)
+            n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_queries and n >= max_queries):
+            break
+    desc = (f"{n} whole decode steps of {wl_name} (sequences {seqs} repeated, cache already resident in host "
+            f"memory), single-threaded C oracle, fp64, {el:.1f} s")
+    return n / el, desc, 1
+
+
+# ---------------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------------
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import workloads as W
+    from workloads import gpu as G
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+    dev = torch.device("cuda", local)
+    wl = W.WORKLOADS[args.workload]
+    B = args.batch or wl.batch
+    step = G.build(args.workload, batch=B, seq_offset=rank * B)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        step.run()
+    barrier()
+
+    # ---- timed region: K steps, per-kernel events on the launching stream ----
+    kern = ("append", "index", "attend") if wl.mode != "prefill" else ("prefill",)
+    ev = {k: [] for k in kern}
+
+    def hook(name, phase):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(stream)
+        if phase == 0:
+            ev[name].append([e, None])
+        else:
+            ev[name][-1][1] = e
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        barrier()
+        torch.cuda._sleep(int(2e7))  # lets the host enqueue the K steps ahead of the GPU
+        start.record(stream)
+        for _ in range(args.steps):
+            if wl.mode == "prefill":
+                hook("prefill", 0)
+                step.run()
+                hook("prefill", 1)
+            else:
+                step.run_parts(hook)
+        end.record(stream)
+        barrier()
+    ms = start.elapsed_time(end)
+    kms = {k: sum(a.elapsed_time(b) for a, b in v) / max(1, len(v)) for k, v in ev.items()}
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    queries_per_step = B * wl.tq * world
+    value = queries_per_step * args.steps / (ms_max / 1e3)
+    launches = args.steps * (len(kern) if wl.mode != "minimal" else 2)
+    if wl.mode == "minimal":
+        kms.pop("index", None)
+
+    # ---- end to end: host inputs -> C ABI call -> host outputs ----
+    e2e = run_e2e(step, args, world, barrier)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_peaks()
+    ab = algorithmic_bytes(wl)
+    dom = "index" if wl.mode in ("full", "reindex") else ("attend" if wl.mode == "minimal" else "prefill")
+    if dom == "prefill":
+        dom_bytes = (ab["index"] + ab["attend"]) * wl.tq
+        dom_file = "index.cu"
+    else:
+        dom_bytes = ab[dom] * B
+        dom_file = "index.cu" if dom == "index" else "attend.cu"
+    dur_s = kms[dom] / 1e3
+    achieved = dom_bytes / dur_s / 1e9
+    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": f"of {peak_kind}",
+            "traffic": ncu_traffic(dom_file, args.workload), "algorithmic_bytes_per_launch": dom_bytes,
+            "ms_per_launch": round(kms[dom], 5)}
+    step_bytes = sum(ab.values()) * B * wl.tq
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (seeded near-Gaussian bf16, sigma 1, clipped to +-26)",
+        "config": {"workload": args.workload, "mode": wl.mode, "batch_per_gpu": B, "context": wl.context,
+                   "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": 16, "head_dim": 128,
+                   "indexer": "4 heads x 64, FP4", "kv_cache": "E2M1 + E4M3/16 (FP4), window FP8",
+                   "window": wl.win, "parallelism": f"dp{world}",
+                   "l2": f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB read per step)",
+                   "step_hbm_gbs": round(step_bytes / (ms_max / args.steps / 1e3) / 1e9, 1),
+                   "accumulate": "fp32 attention, exact fp64 index scores"},
+        "kernel_ms": {k: round(v, 5) for k, v in kms.items()},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        v, desc, cores = oracle_sample(args.workload, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(step, args, world, barrier):
+    import torch
+
+    wl = step.wl
+    if wl.mode == "prefill":
+        names_in = ["kv", "idx_k", "swa_kv", "idx_q", "q"]
+    else:
+        names_in = [n for n in ("qpos", "swa_kv", "idx_q", "q", "pool", "pool_n", "kv", "idx_k", "idx")
+                    if n in step.inputs]
+    host_in = {n: step.inputs[n].cpu().pin_memory() for n in names_in}
+    names_out = ["out"] + (["idx"] if "idx" in step.outputs and wl.mode != "minimal" else [])
+    host_out = {n: torch.empty(step.outputs[n].shape, dtype=step.outputs[n].dtype).pin_memory() for n in names_out}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    stream = torch.cuda.current_stream()
+    K = max(1, args.steps)
+    for _ in range(2):
+        for n, t in host_in.items():
+            step.inputs[n].copy_(t, non_blocking=True)
+        step.run()
+        for n, t in host_out.items():
+            t.copy_(step.outputs[n], non_blocking=True)
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e7))
+    s.record(stream)
+    for _ in range(K):
+        for n, t in host_in.items():
+            step.inputs[n].copy_(t, non_blocking=True)
+        step.run()
+        for n, t in host_out.items():
+            t.copy_(step.outputs[n], non_blocking=True)
+    e.record(stream)
+    barrier()
+    ms = s.elapsed_time(e)
+    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    v = step.batch * wl.tq * world * K / (ms / 1e3)
+    return {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / K, 5), "call": f"csa2_decode_{wl.mode}" if wl.mode != "prefill" else "csa2_prefill_chunk"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, timed on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    v, desc, cores = oracle_sample(args.workload, budget_s=per_step * max(1, args.steps))
+    line = {"metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": args.workload},
+            "cpu_baseline": {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(v, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

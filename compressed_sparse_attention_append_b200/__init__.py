@@ -1,0 +1,260 @@
+"""Thin Python binding of libcsa2 (include/csa2.h): argument marshalling only.
+
+Every function below has the name of the C entry point it calls, takes torch tensors where the C
+call takes device pointers, passes the current CUDA stream, and raises Csa2Error on a non-zero
+status. No step of the CSA2 layer runs here: quantise-append, scoring, Top-k, pool, gather,
+dequantisation and attention all run in the CUDA kernels of libcsa2.so. There is no CPU
+fallback: if the library is not built, loading fails loudly.
+
+Plumbing helpers (`Cache`, `Workspace`) allocate device memory with torch and fill the C structs.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa2.so")
+
+CSA2_OK = 0
+CSA2_ERR_INVALID_ARG = 1
+CSA2_ERR_UNSUPPORTED_SHAPE = 2
+CSA2_ERR_CAPACITY = 3
+CSA2_ERR_WORKSPACE = 4
+CSA2_ERR_CUDA = 5
+CSA2_ERR_DEVICE = 6
+CSA2_DEV_BAD_INDEX = 0x1
+CSA2_DEV_BAD_POS = 0x2
+CSA2_DEV_BAD_POOL = 0x4
+CSA2_SCORE_RELU = 0x1
+
+EXPORTS = (
+    "csa2_entry_bytes", "csa2_status_string", "csa2_version", "csa2_workspace_size", "csa2_workspace_init",
+    "csa2_quantize_append", "csa2_index_topk_full", "csa2_index_topk_reindex", "csa2_sparse_attend",
+    "csa2_decode_full", "csa2_decode_reindex", "csa2_decode_minimal", "csa2_prefill_chunk",
+    "csa2_get_device_status",
+)
+
+
+class Csa2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class csa2_shape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("hq", "d", "hi", "di", "hk", "win", "bs")]
+
+
+class csa2_cache(ctypes.Structure):
+    _fields_ = [
+        ("kv_data", ctypes.c_void_p), ("kv_scale", ctypes.c_void_p), ("ik_data", ctypes.c_void_p),
+        ("ik_scale", ctypes.c_void_p), ("swa", ctypes.c_void_p), ("cap", ctypes.c_int64),
+        ("swa_cap", ctypes.c_int64),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """Load libcsa2.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libcsa2.so is not built at {LIB_PATH}; run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, i64, u32, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t
+        S, C = ctypes.POINTER(csa2_shape), ctypes.POINTER(csa2_cache)
+        sig = {
+            "csa2_entry_bytes": (sz, [i]),
+            "csa2_status_string": (ctypes.c_char_p, [i]),
+            "csa2_version": (i, []),
+            "csa2_workspace_size": (i, [S, i, i, i, i64, i, ctypes.POINTER(sz)]),
+            "csa2_workspace_init": (i, [vp, sz, vp]),
+            "csa2_quantize_append": (i, [S, C, i, i, vp, vp, vp, vp, vp, sz, vp]),
+            "csa2_index_topk_full": (i, [S, C, i, i, vp, vp, i, vp, i, vp, vp, i64, u32, vp, sz, vp]),
+            "csa2_index_topk_reindex": (i, [S, C, i, vp, vp, vp, vp, i, i, vp, u32, vp, sz, vp]),
+            "csa2_sparse_attend": (i, [S, C, i, i, vp, vp, vp, i, vp, f, vp, vp, vp, vp, sz, vp]),
+            "csa2_decode_full": (i, [S, C, i, vp, vp, vp, vp, vp, vp, i, vp, i, vp, vp, i64, vp, f, vp, vp, vp, u32, vp, sz, vp]),
+            "csa2_decode_reindex": (i, [S, C, i, vp, vp, vp, vp, vp, vp, i, i, vp, vp, f, vp, vp, vp, u32, vp, sz, vp]),
+            "csa2_decode_minimal": (i, [S, C, i, vp, vp, vp, vp, i, vp, f, vp, vp, vp, vp, sz, vp]),
+            "csa2_prefill_chunk": (i, [S, C, i64, i, vp, vp, vp, vp, vp, i, vp, i64, f, vp, vp, vp, u32, vp, sz, vp]),
+            "csa2_get_device_status": (i, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().csa2_status_string(int(s)).decode()
+
+
+def _check(fn: str, s: int) -> int:
+    if s != CSA2_OK:
+        raise Csa2Error(fn, s)
+    return s
+
+
+def _p(t):
+    if t is None:
+        return None
+    assert isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous(), "expected a contiguous CUDA tensor"
+    return t.data_ptr()
+
+
+def _bits(t):
+    """bf16 tensors travel as their 16-bit patterns; pointer only."""
+    if t is None:
+        return None
+    assert t.dtype == torch.bfloat16, "expected bf16"
+    return _p(t)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def make_shape(win: int = 128) -> csa2_shape:
+    return csa2_shape(hq=16, d=128, hi=4, di=64, hk=4, win=win, bs=8)
+
+
+class Cache:
+    """Cache planes of `batch` sequences in the layout of include/csa2.h, allocated with torch."""
+
+    def __init__(self, batch: int, cap: int, swa_cap: int = 128, device="cuda", main=True, indexer=True):
+        assert swa_cap & (swa_cap - 1) == 0
+        self.batch, self.cap, self.swa_cap = batch, cap, swa_cap
+        z = lambda *s: torch.zeros(*s, dtype=torch.uint8, device=device)
+        self.kv_data = z(batch, cap, 128) if main else None
+        self.kv_scale = z(batch, cap, 16) if main else None
+        self.ik_data = z(batch, cap, 128) if indexer else None
+        self.ik_scale = z(batch, cap, 16) if indexer else None
+        self.swa = z(batch, swa_cap, 256)
+        self.c = csa2_cache(_p(self.kv_data), _p(self.kv_scale), _p(self.ik_data), _p(self.ik_scale),
+                            _p(self.swa), cap, swa_cap)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def csa2_entry_bytes(channels: int) -> int:
+    return lib().csa2_entry_bytes(int(channels))
+
+
+def csa2_status_string(s: int) -> str:
+    return status_string(s)
+
+
+def csa2_version() -> int:
+    return lib().csa2_version()
+
+
+def csa2_workspace_size(shape, batch, tq, k, max_scan, pool_blocks=0) -> int:
+    out = ctypes.c_size_t(0)
+    _check("csa2_workspace_size", lib().csa2_workspace_size(ctypes.byref(shape), batch, tq, k, max_scan, pool_blocks,
+                                                            ctypes.byref(out)))
+    return out.value
+
+
+def csa2_workspace_init(ws: torch.Tensor, stream=None):
+    _check("csa2_workspace_init", lib().csa2_workspace_init(_p(ws), ws.numel(), _stream(stream)))
+
+
+class Workspace:
+    """A workspace sized by csa2_workspace_size and cleared once by csa2_workspace_init."""
+
+    def __init__(self, shape, batch, tq, k, max_scan, pool_blocks=0, device="cuda", stream=None):
+        n = csa2_workspace_size(shape, batch, tq, k, max_scan, pool_blocks)
+        self.buf = torch.empty(n, dtype=torch.uint8, device=device)
+        assert self.buf.data_ptr() % 256 == 0
+        csa2_workspace_init(self.buf, stream)
+
+    @property
+    def ptr(self):
+        return self.buf.data_ptr()
+
+    @property
+    def nbytes(self):
+        return self.buf.numel()
+
+
+def csa2_quantize_append(shape, cache: Cache, batch, t, pos, kv=None, idx_k=None, swa_kv=None, ws=None, stream=None):
+    _check("csa2_quantize_append", lib().csa2_quantize_append(
+        ctypes.byref(shape), cache.ref, batch, t, _p(pos), _bits(kv), _bits(idx_k), _bits(swa_kv),
+        ws.ptr if ws else None, ws.nbytes if ws else 0, _stream(stream)))
+
+
+def csa2_index_topk_full(shape, cache: Cache, batch, tq, qpos, idx_q, k, out_idx, pool_blocks=0, out_pool=None,
+                         out_pool_n=None, max_ctx=None, flags=0, ws=None, stream=None):
+    if max_ctx is None:
+        max_ctx = cache.cap
+    _check("csa2_index_topk_full", lib().csa2_index_topk_full(
+        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(idx_q), k, _p(out_idx), pool_blocks, _p(out_pool),
+        _p(out_pool_n), max_ctx, flags, ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_index_topk_reindex(shape, cache: Cache, batch, qpos, idx_q, pool, pool_n, k, out_idx, flags=0, ws=None,
+                            stream=None):
+    _check("csa2_index_topk_reindex", lib().csa2_index_topk_reindex(
+        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(idx_q), _p(pool), _p(pool_n), pool.shape[-1], k,
+        _p(out_idx), flags, ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_sparse_attend(shape, cache: Cache, batch, tq, qpos, q, idx, k, out, swa_begin=None, sm_scale=0.0,
+                       out_f32=None, lse=None, ws=None, stream=None):
+    _check("csa2_sparse_attend", lib().csa2_sparse_attend(
+        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
+        _bits(out), _p(out_f32), _p(lse), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_decode_full(shape, cache: Cache, batch, qpos, kv, idx_k, swa_kv, idx_q, q, k, out_idx, out, pool_blocks=0,
+                     out_pool=None, out_pool_n=None, max_ctx=None, swa_begin=None, sm_scale=0.0, out_f32=None,
+                     lse=None, flags=0, ws=None, stream=None):
+    if max_ctx is None:
+        max_ctx = cache.cap
+    _check("csa2_decode_full", lib().csa2_decode_full(
+        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(kv), _bits(idx_k), _bits(swa_kv), _bits(idx_q),
+        _bits(q), k, _p(out_idx), pool_blocks, _p(out_pool), _p(out_pool_n), max_ctx, _p(swa_begin), sm_scale,
+        _bits(out), _p(out_f32), _p(lse), flags, ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_decode_reindex(shape, cache: Cache, batch, qpos, swa_kv, idx_q, q, pool, pool_n, k, out_idx, out,
+                        swa_begin=None, sm_scale=0.0, out_f32=None, lse=None, flags=0, ws=None, stream=None):
+    _check("csa2_decode_reindex", lib().csa2_decode_reindex(
+        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(swa_kv), _bits(idx_q), _bits(q), _p(pool), _p(pool_n),
+        pool.shape[-1], k, _p(out_idx), _p(swa_begin), sm_scale, _bits(out), _p(out_f32), _p(lse), flags, ws.ptr,
+        ws.nbytes, _stream(stream)))
+
+
+def csa2_decode_minimal(shape, cache: Cache, batch, qpos, swa_kv, q, idx, k, out, swa_begin=None, sm_scale=0.0,
+                        out_f32=None, lse=None, ws=None, stream=None):
+    _check("csa2_decode_minimal", lib().csa2_decode_minimal(
+        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(swa_kv), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
+        _bits(out), _p(out_f32), _p(lse), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_prefill_chunk(shape, cache: Cache, pos0, t, kv, idx_k, swa_kv, idx_q, q, k, out_idx, out, swa_begin=0,
+                       sm_scale=0.0, out_f32=None, lse=None, flags=0, ws=None, stream=None):
+    _check("csa2_prefill_chunk", lib().csa2_prefill_chunk(
+        ctypes.byref(shape), cache.ref, pos0, t, _bits(kv), _bits(idx_k), _bits(swa_kv), _bits(idx_q), _bits(q), k,
+        _p(out_idx), swa_begin, sm_scale, _bits(out), _p(out_f32), _p(lse), flags, ws.ptr, ws.nbytes,
+        _stream(stream)))
+
+
+def csa2_get_device_status(ws: Workspace, stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the CSA2_DEV_* bits."""
+    v = ctypes.c_int32(0)
+    s = lib().csa2_get_device_status(ws.ptr, _stream(stream), ctypes.byref(v))
+    if s not in (CSA2_OK, CSA2_ERR_DEVICE):
+        raise Csa2Error("csa2_get_device_status", s)
+    return v.value

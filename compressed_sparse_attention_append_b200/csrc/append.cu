@@ -1,0 +1,131 @@
+// append.cu -- quantise-append of new tokens into the FP4 cache planes and the FP8 window ring.
+//
+// [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token", sec. XI:
+// E2M1 elements with one E4M3 scale per 16 channels and no second-level global scale, quantised
+// after RoPE; the sliding-window KV stays at FP8. [B] "DeepSeek Cuts KV Cache Footprint
+// Fourfold", "Technical Approach": only Full mode writes main KV and indexer keys; every mode
+// writes its own sliding-window KV.
+//
+// Rounding (this build's reading of the unstated rule): s = E4M3_RNE_satfinite(amax / 6) in fp32,
+// all-zero codes when s == 0, code = E2M1_RNE_satfinite(x / s) with the sign of x kept.
+// The quotients are IEEE fp32 divisions; because x has 8 significant bits and s has 4, an fp32
+// quotient can never fall between a rounding boundary and the exact quotient, so these
+// decisions equal those taken on exact rationals.
+//
+// Work split: one thread per 16-channel block. A token has 16 main blocks, hk*4 = 16 indexer
+// blocks and 16 window groups of 16 channels; 48 threads per token.
+#include "csa2_internal.cuh"
+
+namespace csa2 {
+
+namespace {
+
+// Two fp32 -> one byte of two E2M1 codes (first argument -> low nibble), RNE, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "mov.b16 %0, {t, 0};\n\t}"
+        : "=h"(r)
+        : "f"(lo), "f"(hi));
+    return r & 0xFF;
+}
+
+// Two fp32 -> two E4M3 bytes (first argument -> low byte), RNE, saturating to +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&x)[16]) {
+    uint4 a = *reinterpret_cast<const uint4*>(p);
+    uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// One 16-channel block: 8 code bytes + 1 scale byte.
+__device__ __forceinline__ void quantize_block(const float (&x)[16], uint2& codes, uint8_t& scale) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    float s32 = __fdiv_rn(amax, 6.0f);
+    uint32_t sc = f32x2_to_e4m3x2(s32, 0.f) & 0xFF;
+    float s = e4m3_to_f32((uint8_t)sc);
+    uint32_t b[8];
+    if (s == 0.f) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = 0;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = f32x2_to_e2m1x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
+    }
+    codes.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    codes.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    scale = (uint8_t)sc;
+}
+
+__global__ void __launch_bounds__(192) append_kernel(AppendArgs a) {
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long ntok = (long long)a.batch * a.t;
+    if (id >= ntok * 48) return;
+    const long long tok = id / 48;
+    const int task = (int)(id % 48);
+    const int b = (int)(tok / a.t);
+    const int i = (int)(tok % a.t);
+    const int64_t p0 = a.pos ? a.pos[b] : a.pos_host;
+    const int64_t p = p0 + i;
+    if (task < 32) {
+        if (p0 < 0 || p0 + a.t > a.c.cap) {
+            if (task == 0 && i == 0) set_status(a.status, CSA2_DEV_BAD_POS);
+            return;
+        }
+        const bool main = task < 16;
+        const uint16_t* src = main ? a.kv : a.idx_k;
+        if (!src) return;
+        const int blk = main ? task : task - 16;
+        float x[16];
+        load16_bf16(src + tok * 256 + blk * 16, x);
+        uint2 codes;
+        uint8_t sc;
+        quantize_block(x, codes, sc);
+        const size_t row = (size_t)b * a.c.cap + p;
+        uint8_t* dst = main ? a.c.kv_data : a.c.ik_data;
+        uint8_t* sdst = main ? a.c.kv_scale : a.c.ik_scale;
+        *reinterpret_cast<uint2*>(dst + row * 128 + blk * 8) = codes;
+        sdst[row * 16 + blk] = sc;
+    } else {
+        if (!a.swa_kv) return;
+        if (p0 < 0) {
+            if (task == 32 && i == 0) set_status(a.status, CSA2_DEV_BAD_POS);
+            return;
+        }
+        const int g = task - 32;
+        float x[16];
+        load16_bf16(a.swa_kv + tok * 256 + g * 16, x);
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            w[j] = f32x2_to_e4m3x2(x[4 * j], x[4 * j + 1]) | (f32x2_to_e4m3x2(x[4 * j + 2], x[4 * j + 3]) << 16);
+        const size_t slot = (size_t)b * a.c.swa_cap + (size_t)(p & (a.c.swa_cap - 1));
+        *reinterpret_cast<uint4*>(a.c.swa + slot * 256 + g * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
+    const long long threads = (long long)a.batch * a.t * 48;
+    if (threads == 0) return cudaSuccess;
+    const int blk = 192;
+    const long long grid = (threads + blk - 1) / blk;
+    append_kernel<<<(unsigned)grid, blk, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,252 @@
+// csa2_internal.cuh -- device helpers and the workspace plan shared by libcsa2's kernels.
+//
+// Sources (tags as in include/csa2.h):
+//   [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token",
+//       sec. XI "FP4 Main KV Cache": E2M1 elements, one E4M3 scale per 16 channels, no global
+//       scale; SWA KV at FP8.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_fp4.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+// ---- fixed shapes of this build ---------------------------------------------------------------
+constexpr int kHQ = 16;       // query heads
+constexpr int kD = 128;       // head dim (K and V)
+constexpr int kKVBytes = 128; // packed E2M1 bytes of one main K||V row (256 channels)
+constexpr int kKVScales = 16; // E4M3 scale bytes of one main row
+constexpr int kHI = 4;        // indexer query heads
+constexpr int kDI = 64;       // indexer head dim
+constexpr int kHK = 4;        // indexer key heads
+constexpr int kIKBytes = kHK * kDI / 2;   // 128
+constexpr int kIKScales = kHK * kDI / 16; // 16
+constexpr int kBS = 8;        // positions per pool block
+constexpr int kSWABytes = 256;
+constexpr int kMaxK = 2048;   // largest Top-k / pool size
+
+// ---- device status word (first 4 bytes of the workspace) --------------------------------------
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
+    if (status) atomicOr(status, bit);
+}
+
+// ---- codec helpers -----------------------------------------------------------------------------
+// Two E2M1 codes (one byte: low nibble = first element) -> half2 (low half = first element).
+// Hardware conversion cvt.rn.f16x2.e2m1x2 (sm_100a); exact, every E2M1 value is an fp16 value.
+__device__ __forceinline__ void e2m1x8_to_h2x4(uint32_t w, uint32_t (&h)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+}
+
+// Two E4M3 bytes (16-bit: low byte first) -> half2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint16_t v) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+    return r;
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t b) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3);
+    return __half2float(__half(h));
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t h) {
+    __half2 v = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(v);
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+    return __uint_as_float(((uint32_t)b) << 16);
+}
+
+// Orderable 64-bit key of an exact score: larger score <-> larger key; -0 and +0 map to the same
+// key (the score is canonicalised by adding +0).
+__device__ __forceinline__ uint64_t score_key(double s) {
+    s = s + 0.0;
+    uint64_t u = (uint64_t)__double_as_longlong(s);
+    return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// ---- cp.async helpers ----------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+// ---- workspace plan (host and device agree on it) --------------------------------------------------
+struct RowCtr {            // per query row of the index step
+    unsigned int ticket;   // chunk items finished
+    unsigned int ncand;    // candidates emitted
+    unsigned long long tau;// max over finished chunks of their local k-th key (lower bound)
+};
+
+struct IndexPlan {
+    int rows;          // batch * tq
+    int k;
+    int units_max;     // 8-position units scanned per row (upper bound)
+    int chunk_units;   // units per work item
+    int chunks;        // work items per row
+    int pool_blocks;   // 0 = no pool
+    size_t cand_cap;   // candidate slots per row
+};
+
+struct AttendPlan {
+    int rows;
+    int nk_max;        // k + win
+    int kps;           // keys per split (multiple of 64)
+    int splits;
+};
+
+// Workspace: a fixed counter area first (its offsets never depend on the call, so counters
+// left at zero by one call are zero for the next), then per-call data regions.
+//   [0, 256)            header: u32 status, u32 pad, u32 index_next, u32 index_done
+//   [256, +16*kMaxRows) RowCtr per index row
+//   [.., +4*kMaxRows)   attention ticket per row
+//   data: candidates, block maxima, attention partials (contents are scratch)
+constexpr int kMaxRows = 65536;
+constexpr size_t kHdrStatus = 0, kHdrIndexNext = 8, kHdrIndexDone = 12;
+
+struct WsLayout {
+    size_t row_ctr;    // RowCtr[kMaxRows]
+    size_t att_ticket; // u32[kMaxRows]
+    size_t cand_key;   // u64[rows * cand_cap]
+    size_t cand_pos;   // i32[rows * cand_cap]
+    size_t bmax;       // u64[rows * units_max] (pool)
+    size_t att_part;   // f32[rows * splits * hq * (d + 2)]
+    size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline IndexPlan make_index_plan(int rows, int k, int64_t max_scan, int pool_blocks) {
+    IndexPlan p{};
+    p.rows = rows;
+    p.k = k;
+    p.pool_blocks = pool_blocks;
+    p.units_max = (int)((max_scan + kBS - 1) / kBS);
+    if (p.units_max < 1) p.units_max = 1;
+    const int items_target = 148 * 8;
+    int chunks_target = (items_target + rows - 1) / rows;
+    if (chunks_target < 1) chunks_target = 1;
+    int cu = (p.units_max + chunks_target - 1) / chunks_target;
+    cu = (cu + 31) / 32 * 32;
+    if (cu < 32) cu = 32;
+    if (cu > 2048) cu = 2048;
+    p.chunk_units = cu;
+    p.chunks = (p.units_max + cu - 1) / cu;
+    p.cand_cap = (size_t)p.chunks * (size_t)k;
+    return p;
+}
+
+inline AttendPlan make_attend_plan(int rows, int k, int win) {
+    AttendPlan a{};
+    a.rows = rows;
+    a.nk_max = k + win;
+    int tiles = (a.nk_max + 63) / 64;
+    int splits = (2 * 148 + rows - 1) / rows;
+    if (splits < 1) splits = 1;
+    if (splits > tiles) splits = tiles;
+    a.kps = ((tiles + splits - 1) / splits) * 64;
+    a.splits = (a.nk_max + a.kps - 1) / a.kps;
+    return a;
+}
+
+inline WsLayout make_layout(const IndexPlan* ip, const AttendPlan* ap) {
+    WsLayout L{};
+    size_t off = 256;
+    L.row_ctr = off; off = align256(off + sizeof(RowCtr) * (size_t)kMaxRows);
+    L.att_ticket = off; off = align256(off + 4 * (size_t)kMaxRows);
+    int rows_i = ip ? ip->rows : 0;
+    size_t cc = ip ? ip->cand_cap : 0;
+    L.cand_key = off; off = align256(off + 8 * (size_t)rows_i * cc);
+    L.cand_pos = off; off = align256(off + 4 * (size_t)rows_i * cc);
+    size_t bm = (ip && ip->pool_blocks > 0) ? (size_t)rows_i * (size_t)ip->units_max : 0;
+    L.bmax = off; off = align256(off + 8 * bm);
+    size_t part = ap ? (size_t)ap->rows * (size_t)ap->splits * kHQ * (kD + 2) : 0;
+    L.att_part = off; off = align256(off + 4 * part);
+    L.total = off;
+    return L;
+}
+
+// ---- kernel launchers (defined in append.cu, index.cu, attend.cu) -----------------------------------
+struct AppendArgs {
+    csa2_cache c;
+    int batch, t;
+    const int64_t* pos;  // [batch], or NULL: every sequence starts at pos_host
+    int64_t pos_host;
+    const uint16_t* kv;
+    const uint16_t* idx_k;
+    const uint16_t* swa_kv;
+    uint32_t* status;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+
+struct IndexArgs {
+    csa2_cache c;
+    int rows;            // batch * tq
+    int tq;
+    const int64_t* qpos; // [rows], or NULL: row r sits at qpos_base + r % tq
+    int64_t qpos_base;
+    const uint16_t* idx_q;
+    int reindex;         // 0 = Full, 1 = Reindex
+    const int32_t* pool; // Reindex: [batch][pool_stride]
+    const int32_t* pool_n;
+    int pool_stride;
+    int64_t max_ctx;     // Full: bound on qpos+1
+    int32_t* out_idx;
+    int32_t* out_pool;
+    int32_t* out_pool_n;
+    uint32_t flags;
+    IndexPlan plan;
+    unsigned char* ws;
+    WsLayout L;
+};
+cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);
+
+struct AttendArgs {
+    csa2_cache c;
+    int rows, tq, k, win;
+    const int64_t* qpos;  // or NULL: qpos_base + r % tq
+    int64_t qpos_base;
+    int64_t swa_begin_host;  // used when swa_begin is NULL
+    const uint16_t* q;
+    const int32_t* idx;
+    const int64_t* swa_begin;
+    float sm_scale;
+    uint16_t* out;
+    float* out_f32;
+    float* lse;
+    AttendPlan plan;
+    unsigned char* ws;
+    WsLayout L;
+};
+cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
+
+}  // namespace csa2

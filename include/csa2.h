@@ -1,0 +1,247 @@
+/*
+ * csa2.h -- C ABI of libcsa2: one CSA2 (Compressed Sparse Attention 2) layer step over an FP4
+ * KV cache, on one NVIDIA B200 (sm_100a).
+ *
+ * Sources (tags used in the comments below):
+ *   [A] "DeepSeek-V4.1-Flash: Shrinking KV Cache at 552B Scale" (visualisation captions page)
+ *   [B] "DeepSeek Cuts KV Cache Footprint Fourfold" (paper summary), "Technical Approach"
+ *   [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token"
+ *       (engineering article), sections VI, VII, IX, XI, XII
+ *
+ * The pages define the operations but no API, no cache layout, no index-score formula, no
+ * softmax scale and no rounding rule. Where this header fixes one of those, it says so.
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless marked "host". bf16 tensors are passed as their raw
+ *     16-bit patterns (uint16_t). All tensors are dense, row-major, in the shapes stated.
+ *   - Ownership: the caller owns every buffer (cache planes, inputs, outputs, workspace).
+ *     libcsa2 allocates nothing, keeps no mutable global state and never frees.
+ *   - Streams: `stream` is a cudaStream_t passed as void*. Every call only enqueues work on it
+ *     and returns without synchronising (except csa2_get_device_status). Calls on one stream
+ *     run in order; calls that share one workspace must not run concurrently.
+ *   - Errors: host-checkable argument errors return a status before anything is enqueued.
+ *     Errors found on the device (an inherited index out of range, an append past the cache
+ *     capacity, a pool block id out of range) set bits of a status word inside the workspace
+ *     and the offending item is skipped; read it with csa2_get_device_status. No call traps,
+ *     asserts or spins on the device.
+ *   - Fixed shapes of this build: hq = 16 query heads, d = 128 (K and V each), one shared KV
+ *     head, hi = 4 indexer query heads, di = 64, hk = 4 indexer key heads, bs = 8 positions
+ *     per pool block, win <= 128. Other values return CSA2_ERR_UNSUPPORTED_SHAPE.
+ */
+#ifndef CSA2_H
+#define CSA2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define CSA2_API __attribute__((visibility("default")))
+#else
+#define CSA2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA2_OK = 0,
+    CSA2_ERR_INVALID_ARG = 1,      /* null pointer, negative size, misaligned pointer        */
+    CSA2_ERR_UNSUPPORTED_SHAPE = 2,/* shape outside what this build implements               */
+    CSA2_ERR_CAPACITY = 3,         /* a bound that the host can see exceeds the cache        */
+    CSA2_ERR_WORKSPACE = 4,        /* workspace pointer null or smaller than required        */
+    CSA2_ERR_CUDA = 5,             /* a kernel launch failed (cudaGetLastError)              */
+    CSA2_ERR_DEVICE = 6            /* csa2_get_device_status found device-side error bits    */
+} csa2_status;
+
+/* Device status bits (csa2_get_device_status). */
+#define CSA2_DEV_BAD_INDEX   0x1   /* selected / inherited index < -1, > qpos or >= cap       */
+#define CSA2_DEV_BAD_POS     0x2   /* append position outside [0, cap) or qpos >= bound       */
+#define CSA2_DEV_BAD_POOL    0x4   /* pool block id outside [0, cap / bs)                     */
+
+/* Flags for the index entry points. */
+#define CSA2_SCORE_RELU      0x1u  /* score = sum_h max(0, q_h . k_h) instead of sum_h q_h . k_h */
+
+typedef struct {
+    int hq;   /* query heads (16)                                 */
+    int d;    /* head dim of K and of V (128)                     */
+    int hi;   /* indexer query heads (4)                          */
+    int di;   /* indexer head dim (64)                            */
+    int hk;   /* indexer key heads (4)                            */
+    int win;  /* sliding-window length (128; [C] config list)     */
+    int bs;   /* positions per pool block (8; [C] sec. IX)        */
+} csa2_shape;
+
+/*
+ * Cache of `batch` sequences (layout fixed by this build; the pages give none). Per sequence b
+ * and position p (0 <= p < cap):
+ *   kv_data  + (b*cap + p)*128      : main K||V, 256 channels (K = 0..127, V = 128..255) as E2M1
+ *                                     codes, channel 2j in the low nibble of byte j
+ *   kv_scale + (b*cap + p)*16       : one E4M3 scale byte per 16 channels (block b <-> byte b)
+ *   ik_data  + (b*cap + p)*hk*32    : indexer key, hk heads x 64 channels, E2M1 as above
+ *   ik_scale + (b*cap + p)*hk*4     : its E4M3 scales
+ *   swa      + (b*swa_cap + (p & (swa_cap-1)))*256 : sliding-window K||V as E4M3 bytes (no
+ *                                     scale), a ring of swa_cap slots (power of two)
+ * Every plane base must be 16-byte aligned. Entry bytes: 144 (main) + 144 (indexer) per
+ * position; csa2_entry_bytes gives the rule.
+ */
+typedef struct {
+    uint8_t* kv_data;
+    uint8_t* kv_scale;
+    uint8_t* ik_data;
+    uint8_t* ik_scale;
+    uint8_t* swa;
+    int64_t cap;      /* positions per sequence in the main and indexer planes */
+    int64_t swa_cap;  /* ring slots per sequence, power of two, >= win (decode) */
+} csa2_cache;
+
+/* [C] sec. VII (byte budget): an entry of `channels` E2M1 values with one 1-byte E4M3 scale per
+ * 16 channels occupies channels/2 + channels/16 bytes. Returns 0 if channels is not a positive
+ * multiple of 16. Host only. */
+CSA2_API size_t csa2_entry_bytes(int channels);
+
+/* Text of a status code. Host only; never NULL. */
+CSA2_API const char* csa2_status_string(csa2_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. Host only. */
+CSA2_API int csa2_version(void);
+
+/*
+ * Workspace bytes needed by any entry point below when called with at most `batch` sequences,
+ * `tq` query rows per sequence, top-k `k` (<= 2048), at most `max_scan` positions scanned by
+ * the indexer per query row (Full: the largest qpos+1; Reindex: pool entries * bs) and
+ * `pool_blocks` pool blocks (0 if no pool is built). Host only. The workspace must be 256-byte
+ * aligned and, once after allocation, cleared with csa2_workspace_init; every call leaves its
+ * counters cleared again.
+ */
+CSA2_API csa2_status csa2_workspace_size(const csa2_shape* shape, int batch, int tq, int k, int64_t max_scan,
+                                int pool_blocks, size_t* bytes /* host */);
+
+/* Zeroes the workspace (one cudaMemsetAsync on `stream`). */
+CSA2_API csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Quantise-append. [C] sec. XI: cached values are E2M1 with one E4M3 scale per 16 channels and
+ * no second-level global scale, quantised after RoPE; the sliding-window KV stays at FP8.
+ * [B] "Technical Approach": Full mode writes main KV and indexer keys, Reindex and Minimal
+ * write only their own sliding-window KV (pass NULL for the planes a mode does not write).
+ *   pos    [batch] int64 : first new position of each sequence; tokens go to pos..pos+t-1
+ *   kv     [batch][t][256] bf16 or NULL  -> kv_data / kv_scale
+ *   idx_k  [batch][t][hk*64] bf16 or NULL -> ik_data / ik_scale
+ *   swa_kv [batch][t][256] bf16 or NULL  -> swa ring slots (pos+i) & (swa_cap-1)
+ * Rounding (this build's reading): per 16-channel block s = E4M3_RNE_satfinite(amax/6);
+ * s == 0 gives all-zero codes; code_i = E2M1_RNE_satfinite(x_i / s) keeping the sign of x_i;
+ * SWA bytes = E4M3_RNE_satfinite(x). A sequence whose range leaves [0, cap) sets
+ * CSA2_DEV_BAD_POS and is skipped (needs `ws`; pass NULL to skip the device check).
+ */
+CSA2_API csa2_status csa2_quantize_append(const csa2_shape* shape, const csa2_cache* cache, int batch, int t,
+                                 const int64_t* pos, const uint16_t* kv, const uint16_t* idx_k,
+                                 const uint16_t* swa_kv, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Full-mode index step. [B] "Technical Approach": Full mode computes the Top-K indices;
+ * [C] sec. VI "Shortlist-of-a-shortlist" and sec. IX Figure 4: the decoder's first Full layer
+ * scores every causally visible position, and collects the blocks with the highest maximum
+ * score (up to 2,048 blocks of 8 positions) into a shared candidate pool.
+ *   qpos     [batch*tq] int64 : query position of each row; positions 0..qpos are visible
+ *   idx_q    [batch][tq][hi][di] bf16 : indexer query, quantised in-kernel with the codec above
+ *   k        : Top-k (<= 2048)
+ *   out_idx  [batch][tq][k] int32 : selected positions, ascending, padded with -1
+ *   pool_blocks : 0, or the pool size P (decode only: tq == 1)
+ *   out_pool [batch][P] int32 : pool block ids, ascending, padded with -1 (NULL if P == 0)
+ *   out_pool_n [batch] int32 : min(P, ceil((qpos+1)/bs))          (NULL if P == 0)
+ *   max_ctx  : host upper bound on qpos+1 over all rows (<= cap)
+ * Score (this build's reading): score(p) = sum_h q_h . k_{p,h} on dequantised values, exact;
+ * ranking by score descending, ties to the lower position (lower block id for the pool).
+ */
+CSA2_API csa2_status csa2_index_topk_full(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
+                                 const int64_t* qpos, const uint16_t* idx_q, int k, int32_t* out_idx,
+                                 int pool_blocks, int32_t* out_pool, int32_t* out_pool_n, int64_t max_ctx,
+                                 uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Reindex-mode index step (decode, one query row per sequence). [B] "Technical Approach" and
+ * [C] sec. VI: a fresh indexer query chooses its Top-k only inside the shared candidate pool.
+ *   qpos   [batch] int64, idx_q [batch][hi][di] bf16
+ *   pool   [batch][pool_stride] int32 : block ids (each covers positions bs*id .. bs*id+bs-1)
+ *   pool_n [batch] int32 : entries used in each row (<= pool_stride)
+ *   out_idx [batch][k] int32 : ascending, padded with -1; positions > qpos are never chosen
+ */
+CSA2_API csa2_status csa2_index_topk_reindex(const csa2_shape* shape, const csa2_cache* cache, int batch,
+                                    const int64_t* qpos, const uint16_t* idx_q, const int32_t* pool,
+                                    const int32_t* pool_n, int pool_stride, int k, int32_t* out_idx,
+                                    uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse attention. [C] sec. VI "What one layer looks like": the layer's own query attends to
+ * the selected entries of the shared main KV plus its own recent window; [C] sec. XI: cached
+ * values are dequantised before attention; [C] sec. XII: with a replay start s, a query at i
+ * sees window keys [max(s, i-win+1), i].
+ *   qpos [batch*tq] int64, q [batch][tq][hq][d] bf16
+ *   idx  [batch][tq][k] int32 : main-KV positions, -1 = skip, any order
+ *   swa_begin [batch] int64 or NULL (= 0)
+ *   sm_scale : softmax scale, 0 gives 1/sqrt(d)
+ *   out [batch][tq][hq][d] bf16; out_f32 (same shape, fp32) and lse [batch][tq][hq] fp32 (natural
+ *   log) may be NULL.
+ * This build's reading: ONE softmax over selected rows and window rows together; a position may
+ * appear in both (its FP4 main entry and its FP8 window entry are different vectors). An index
+ * < -1, > qpos or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row with no key gives out = 0
+ * and lse = -inf.
+ */
+CSA2_API csa2_status csa2_sparse_attend(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
+                               const int64_t* qpos, const uint16_t* q, const int32_t* idx, int k,
+                               const int64_t* swa_begin, float sm_scale, uint16_t* out, float* out_f32,
+                               float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One decode step per mode ([B] "Technical Approach": Full computes main KV, indexer keys and
+ * Top-K; Reindex reuses main KV and indexer keys and recomputes the selection; Minimal reuses
+ * all three and computes only its own query and sliding-window KV). Each is the composition
+ * quantise-append -> index step -> sparse attention on `stream`, with the arguments above;
+ * the new token sits at qpos[b] (appended before scoring, so it is visible).
+ *   decode_full    : appends kv, idx_k, swa_kv; Full index step (pool optional); attention
+ *   decode_reindex : appends swa_kv; Reindex index step; attention
+ *   decode_minimal : appends swa_kv; attention with the inherited idx
+ */
+CSA2_API csa2_status csa2_decode_full(const csa2_shape* shape, const csa2_cache* cache, int batch, const int64_t* qpos,
+                             const uint16_t* kv, const uint16_t* idx_k, const uint16_t* swa_kv,
+                             const uint16_t* idx_q, const uint16_t* q, int k, int32_t* out_idx,
+                             int pool_blocks, int32_t* out_pool, int32_t* out_pool_n, int64_t max_ctx,
+                             const int64_t* swa_begin, float sm_scale, uint16_t* out, float* out_f32,
+                             float* lse, uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+CSA2_API csa2_status csa2_decode_reindex(const csa2_shape* shape, const csa2_cache* cache, int batch,
+                                const int64_t* qpos, const uint16_t* swa_kv, const uint16_t* idx_q,
+                                const uint16_t* q, const int32_t* pool, const int32_t* pool_n,
+                                int pool_stride, int k, int32_t* out_idx, const int64_t* swa_begin,
+                                float sm_scale, uint16_t* out, float* out_f32, float* lse, uint32_t flags,
+                                void* ws, size_t ws_bytes, void* stream);
+
+CSA2_API csa2_status csa2_decode_minimal(const csa2_shape* shape, const csa2_cache* cache, int batch,
+                                const int64_t* qpos, const uint16_t* swa_kv, const uint16_t* q,
+                                const int32_t* idx, int k, const int64_t* swa_begin, float sm_scale,
+                                uint16_t* out, float* out_f32, float* lse, void* ws, size_t ws_bytes,
+                                void* stream);
+
+/*
+ * Prefill chunk of t tokens at positions pos0..pos0+t-1 of one sequence (batch 1). [C] sec. X
+ * and XI: the chunk's K/V and indexer keys are quantised and appended; every new token then
+ * selects its Top-k among positions <= its own and attends to them plus its window.
+ *   kv [t][256], idx_k [t][hk*64], swa_kv [t][256], idx_q [t][hi][di], q [t][hq][d] (bf16)
+ *   out_idx [t][k] int32, out [t][hq][d] bf16; swa_cap must be >= t + win.
+ */
+CSA2_API csa2_status csa2_prefill_chunk(const csa2_shape* shape, const csa2_cache* cache, int64_t pos0, int t,
+                               const uint16_t* kv, const uint16_t* idx_k, const uint16_t* swa_kv,
+                               const uint16_t* idx_q, const uint16_t* q, int k, int32_t* out_idx,
+                               int64_t swa_begin, float sm_scale, uint16_t* out, float* out_f32, float* lse,
+                               uint32_t flags, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device status word in `ws`.
+ * *host_status receives the CSA2_DEV_* bits; returns CSA2_ERR_DEVICE if any bit was set. */
+CSA2_API csa2_status csa2_get_device_status(void* ws, void* stream, int32_t* host_status /* host */);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA2_H */

@@ -1,0 +1,131 @@
+"""The C-ABI library loads and exports every symbol include/csa2.h declares; host-only calls and
+argument validation (which returns before anything touches a GPU) behave as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import compressed_sparse_attention_append_b200 as csa
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def L():
+    from compressed_sparse_attention_append_b200 import build
+
+    build.build()
+    return csa.lib()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    return re.findall(r"CSA2_API\s+[\w\s\*]+?\b(csa2_\w+)\s*\(", src)
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) == 14
+    assert set(names) == set(csa.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_header_compiles_as_c():
+    import subprocess
+    import tempfile
+
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        with open(c, "w") as f:
+            f.write('#include "csa2.h"\nint main(void){ csa2_shape s; csa2_cache c; (void)s; (void)c; return 0; }\n')
+        subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-c", c,
+                               "-o", os.path.join(d, "t.o")])
+
+
+def test_host_functions(L):
+    assert csa.csa2_entry_bytes(256) == 144
+    assert csa.csa2_entry_bytes(512) == 288
+    assert csa.csa2_entry_bytes(24) == 0 and csa.csa2_entry_bytes(-16) == 0
+    assert csa.csa2_version() == 100
+    for s in range(7):
+        assert csa.csa2_status_string(s)
+    assert csa.csa2_status_string(99) == "unknown status"
+
+
+def test_workspace_size_is_monotone_and_validates(L):
+    sh = csa.make_shape()
+    a = csa.csa2_workspace_size(sh, 128, 1, 512, 16000, 0)
+    b = csa.csa2_workspace_size(sh, 64, 1, 512, 131072, 2048)
+    assert a > 0 and b > a // 4
+    assert csa.csa2_workspace_size(sh, 1, 1, 512, 4096) >= 256
+    bad = csa.make_shape()
+    bad.hq = 8
+    with pytest.raises(csa.Csa2Error) as e:
+        csa.csa2_workspace_size(bad, 1, 1, 512, 4096)
+    assert e.value.status == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    with pytest.raises(csa.Csa2Error) as e:
+        csa.csa2_workspace_size(sh, 1, 1, 4096, 4096)
+    assert e.value.status == csa.CSA2_ERR_INVALID_ARG
+
+
+def _fake_cache(cap=4096, swa_cap=128, align=16):
+    base = 1 << 40
+    return csa.csa2_cache(base, base + 1 * align * 1024, base + 2 * align * 1024, base + 3 * align * 1024,
+                          base + 4 * align * 1024, cap, swa_cap)
+
+
+def test_validation_before_launch(L):
+    """Each call below must return its error without launching (the pointers are not real)."""
+    sh = csa.make_shape()
+    c = _fake_cache()
+    F = 1 << 41
+    vp = F
+    # unsupported shape
+    bad = csa.make_shape()
+    bad.di = 32
+    assert L.csa2_index_topk_full(ctypes.byref(bad), ctypes.byref(c), 1, 1, vp, vp, 512, vp, 0, None, None, 100, 0,
+                                  vp, 1 << 30, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    # k out of range / pool with tq > 1 / max_ctx beyond capacity / unknown flag
+    assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 1, 1, vp, vp, 0, vp, 0, None, None, 100, 0, vp,
+                                  1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 1, 2, vp, vp, 512, vp, 64, vp, vp, 100, 0, vp,
+                                  1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 1, 1, vp, vp, 512, vp, 0, None, None, 5000, 0,
+                                  vp, 1 << 30, None) == csa.CSA2_ERR_CAPACITY
+    assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 1, 1, vp, vp, 512, vp, 0, None, None, 100, 8,
+                                  vp, 1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    # workspace too small / missing
+    assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 4, 1, vp, vp, 512, vp, 0, None, None, 4096, 0,
+                                  vp, 1024, None) == csa.CSA2_ERR_WORKSPACE
+    assert L.csa2_sparse_attend(ctypes.byref(sh), ctypes.byref(c), 4, 1, vp, vp, vp, 512, None, 0.0, vp, None, None,
+                                None, 0, None) == csa.CSA2_ERR_WORKSPACE
+    # misaligned pointer, bad ring capacity, NaN scale
+    assert L.csa2_sparse_attend(ctypes.byref(sh), ctypes.byref(c), 4, 1, vp, vp + 2, vp, 512, None, 0.0, vp, None,
+                                None, vp, 1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    c2 = _fake_cache(swa_cap=100)
+    assert L.csa2_sparse_attend(ctypes.byref(sh), ctypes.byref(c2), 4, 1, vp, vp, vp, 512, None, 0.0, vp, None, None,
+                                vp, 1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    assert L.csa2_sparse_attend(ctypes.byref(sh), ctypes.byref(c), 4, 1, vp, vp, vp, 512, None, float("nan"), vp, None,
+                                None, vp, 1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    # append beyond capacity (host-visible), null pos
+    assert L.csa2_quantize_append(ctypes.byref(sh), ctypes.byref(c), 1, 5000, vp, vp, None, None, None, 0,
+                                  None) == csa.CSA2_ERR_CAPACITY
+    assert L.csa2_quantize_append(ctypes.byref(sh), ctypes.byref(c), 1, 1, None, vp, None, None, None, 0,
+                                  None) == csa.CSA2_ERR_INVALID_ARG
+    # prefill: window ring too small for the chunk
+    assert L.csa2_prefill_chunk(ctypes.byref(sh), ctypes.byref(c), 0, 256, vp, vp, vp, vp, vp, 512, vp, 0, 0.0, vp,
+                                None, None, 0, vp, 1 << 30, None) == csa.CSA2_ERR_CAPACITY
+    # device status needs a workspace
+    v = ctypes.c_int32(0)
+    assert L.csa2_get_device_status(None, None, ctypes.byref(v)) == csa.CSA2_ERR_INVALID_ARG
+
+
+def test_product_path_has_no_oracle_dependency():
+    """The package and the kernels never import, link or read the oracle."""
+    pkg = os.path.join(ROOT, "compressed_sparse_attention_append_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in txt.lower(), f

@@ -1,0 +1,134 @@
+"""Index scoring, exact Top-k, block pool and Reindex on the GPU against the oracle: index sets
+must be identical (the scores are exact on both sides and the ranking is a total order)."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_attention_append_b200 as csa
+import oracle
+import workloads as W
+from _gpu import DEV, bf16_np, gpu_fill, oracle_seq, query_values, values
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(B, n, seed, sigma=1.0, cap=None):
+    cap = cap or n
+    shape = csa.make_shape()
+    swa_cap = 1 << max(7, (n - 1).bit_length())
+    cache = csa.Cache(B, cap, swa_cap)
+    gpu_fill(cache, shape, seed, B, n, sigma)
+    return shape, cache, swa_cap
+
+
+@pytest.mark.parametrize("B,n,k,pool,sigma,ragged", [
+    (1, 37, 16, 4, 1.0, False),
+    (3, 600, 64, 16, 1.0, True),
+    (2, 4099, 512, 0, 1.0, True),
+    (2, 9000, 512, 2048, 8.0, True),
+    (1, 20000, 512, 600, 1.0, False),
+])
+def test_full_mode_matches_oracle(orc, B, n, k, pool, sigma, ragged):
+    seed = 11 + n
+    shape, cache, swa_cap = _setup(B, n, seed, sigma)
+    qpos = [n - 1 - (37 * i if ragged else 0) for i in range(B)]
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV)
+    iq = query_values(seed, "iq", torch.arange(B), qp, 256, DEV, sigma).contiguous()
+    out = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
+    opool = torch.full((B, max(pool, 1)), -7, dtype=torch.int32, device=DEV)
+    opn = torch.zeros(B, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, n, pool)
+    refs = []
+    for b in range(B):
+        oc = oracle_seq(seed, b, n, n, swa_cap, sigma)
+        qb = query_values(seed, "iq", [b], [qpos[b]], 256, "cpu", sigma)[0]
+        refs.append(oc.index_topk_full(qpos[b], qb, k=k, pool_blocks=pool) if pool else
+                    (oc.index_topk_full(qpos[b], qb, k=k), None, None))
+    for rep in range(2):  # the second call checks that the counters were left cleared
+        csa.csa2_index_topk_full(shape, cache, B, 1, qp, iq, k, out, pool, opool if pool else None,
+                                 opn if pool else None, max_ctx=n, ws=ws)
+        assert csa.csa2_get_device_status(ws) == 0
+        for b in range(B):
+            ridx, rpool, rpn = refs[b]
+            if pool:
+                assert int(opn[b]) == rpn
+                assert np.array_equal(opool[b].cpu().numpy(), rpool)
+            assert np.array_equal(out[b].cpu().numpy(), ridx), (rep, b)
+
+
+def test_full_mode_relu_and_ties(orc):
+    """Identical indexer keys at many positions force exact score ties: the lower position wins."""
+    B, n, k = 1, 3000, 512
+    shape = csa.make_shape()
+    cache = csa.Cache(B, n, 4096)
+    p = torch.arange(n, device=DEV)
+    ik = values(3, "ik", [0], p % 97, 256, DEV).contiguous()  # 97 distinct keys, repeated
+    kv = values(3, "kv", [0], p, 256, DEV).contiguous()
+    csa.csa2_quantize_append(shape, cache, 1, n, torch.zeros(1, dtype=torch.int64, device=DEV), kv, ik, kv)
+    iq = query_values(3, "iq", [0], [n - 1], 256, DEV).contiguous()
+    qp = torch.tensor([n - 1], dtype=torch.int64, device=DEV)
+    oc = oracle.SeqCache(n, 4096)
+    oc.append(0, kv=bf16_np(kv[0]), idx_k=bf16_np(ik[0]))
+    qb = bf16_np(iq[0])
+    for flags, relu in ((0, False), (csa.CSA2_SCORE_RELU, True)):
+        out = torch.empty(B, k, dtype=torch.int32, device=DEV)
+        ws = csa.Workspace(shape, B, 1, k, n)
+        csa.csa2_index_topk_full(shape, cache, B, 1, qp, iq, k, out, max_ctx=n, flags=flags, ws=ws)
+        ref = oc.index_topk_full(n - 1, qb, k=k, relu=relu)
+        assert np.array_equal(out[0].cpu().numpy(), ref), relu
+
+
+@pytest.mark.parametrize("B,n,P,k", [(2, 4096, 40, 128), (3, 50000, 2000, 512), (1, 1000, 125, 512)])
+def test_reindex_matches_oracle(orc, B, n, P, k):
+    seed = 23 + P
+    shape, cache, swa_cap = _setup(B, n, seed)
+    nblk = (n + 7) // 8
+    pool = W.distinct_sorted(seed, "pool", torch.arange(B, device=DEV), nblk, P).to(torch.int32).contiguous()
+    pool_n = torch.tensor([P - 3 * i for i in range(B)], dtype=torch.int32, device=DEV)
+    qpos = [n - 1 - 101 * i for i in range(B)]
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV)
+    iq = query_values(seed, "iq", torch.arange(B), qp, 256, DEV).contiguous()
+    out = torch.full((B, k), -7, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, P * 8)
+    csa.csa2_index_topk_reindex(shape, cache, B, qp, iq, pool, pool_n, k, out, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    for b in range(B):
+        oc = oracle_seq(seed, b, n, n, swa_cap)
+        qb = query_values(seed, "iq", [b], [qpos[b]], 256, "cpu")[0]
+        pl = pool[b].cpu().numpy()
+        ref = oc.index_topk_reindex(qpos[b], qb, pl, int(pool_n[b]), k=k)
+        assert np.array_equal(out[b].cpu().numpy(), ref), b
+
+
+def test_reindex_with_full_query_reproduces_full_topk(orc):
+    """Pool built by Full mode, then Reindex with the same query: the same Top-k."""
+    B, n, k, P = 2, 30000, 512, 2048
+    shape, cache, _ = _setup(B, n, 77)
+    qp = torch.tensor([n - 1, n - 500], dtype=torch.int64, device=DEV)
+    iq = query_values(77, "iq", torch.arange(B), qp, 256, DEV).contiguous()
+    out = torch.empty(B, k, dtype=torch.int32, device=DEV)
+    opool = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    opn = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, n, P)
+    csa.csa2_index_topk_full(shape, cache, B, 1, qp, iq, k, out, P, opool, opn, max_ctx=n, ws=ws)
+    out2 = torch.empty(B, k, dtype=torch.int32, device=DEV)
+    csa.csa2_index_topk_reindex(shape, cache, B, qp, iq, opool, opn, k, out2, ws=ws)
+    assert torch.equal(out, out2)
+    for b in range(B):
+        sel = out[b][out[b] >= 0]
+        blocks = set(opool[b][: int(opn[b])].tolist())
+        assert all(int(x) // 8 in blocks for x in sel)
+
+
+def test_bad_pool_id_sets_status():
+    shape, cache, _ = _setup(1, 256, 5)
+    pool = torch.tensor([[0, 3, 1000]], dtype=torch.int32, device=DEV)
+    pool_n = torch.tensor([3], dtype=torch.int32, device=DEV)
+    qp = torch.tensor([255], dtype=torch.int64, device=DEV)
+    iq = query_values(5, "iq", [0], qp, 256, DEV).contiguous()
+    out = torch.empty(1, 16, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, 1, 1, 16, 24)
+    csa.csa2_index_topk_reindex(shape, cache, 1, qp, iq, pool, pool_n, 16, out, ws=ws)
+    assert csa.csa2_get_device_status(ws) == csa.CSA2_DEV_BAD_POOL
+    got = out[0].cpu().numpy()
+    assert set(got[got >= 0].tolist()) == set(range(0, 8)) | set(range(24, 32))

@@ -1,0 +1,187 @@
+"""Builds the five workloads on a GPU through libcsa2's C ABI (bench.py and the full-size parity
+tests use it). Inputs come from the seeded generator in workloads/__init__.py, made on the device;
+the cache is filled with libcsa2's own quantise-append. Only the positions a step can read are
+filled (a Reindex step reads only its pool, a Minimal step only its inherited rows); the rest of
+each allocated plane stays zero.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import torch
+
+import compressed_sparse_attention_append_b200 as csa
+from . import WORKLOADS, Workload, cache_values, distinct_sorted
+
+
+def _vals(seed, stream, b, p, width):
+    return cache_values(seed, stream, b, p, width)
+
+
+@dataclasses.dataclass
+class Step:
+    wl: Workload
+    shape: object
+    cache: csa.Cache
+    ws: csa.Workspace
+    inputs: dict            # per-step device inputs
+    outputs: dict           # per-step device outputs
+    batch: int
+    max_ctx: int
+
+    # ---- one pass of the hot path, through the composed entry point ----
+    def run(self, stream=None, ws=None, out_f32=None, lse=None):
+        wl, I, O = self.wl, self.inputs, self.outputs
+        ws = ws or self.ws
+        if wl.mode == "full":
+            csa.csa2_decode_full(self.shape, self.cache, self.batch, I["qpos"], I["kv"], I["idx_k"], I["swa_kv"],
+                                 I["idx_q"], I["q"], wl.k, O["idx"], O["out"], pool_blocks=wl.pool_blocks,
+                                 out_pool=O.get("pool"), out_pool_n=O.get("pool_n"), max_ctx=self.max_ctx,
+                                 out_f32=out_f32, lse=lse, ws=ws, stream=stream)
+        elif wl.mode == "reindex":
+            csa.csa2_decode_reindex(self.shape, self.cache, self.batch, I["qpos"], I["swa_kv"], I["idx_q"], I["q"],
+                                    I["pool"], I["pool_n"], wl.k, O["idx"], O["out"], out_f32=out_f32, lse=lse,
+                                    ws=ws, stream=stream)
+        elif wl.mode == "minimal":
+            csa.csa2_decode_minimal(self.shape, self.cache, self.batch, I["qpos"], I["swa_kv"], I["q"], I["idx"],
+                                    wl.k, O["out"], out_f32=out_f32, lse=lse, ws=ws, stream=stream)
+        else:
+            csa.csa2_prefill_chunk(self.shape, self.cache, wl.context - wl.tq, wl.tq, I["kv"], I["idx_k"],
+                                   I["swa_kv"], I["idx_q"], I["q"], wl.k, O["idx"], O["out"], out_f32=out_f32,
+                                   lse=lse, ws=ws, stream=stream)
+
+    # ---- the same pass as separate entry points (kernel-level timing) ----
+    def run_parts(self, hooks, stream=None):
+        """hooks(name) is called before and after each kernel's entry point: ('append'|'index'|'attend')."""
+        wl, I, O = self.wl, self.inputs, self.outputs
+        b = self.batch
+        if wl.mode == "prefill":
+            raise NotImplementedError("prefill is timed through csa2_prefill_chunk")
+        hooks("append", 0)
+        if wl.mode == "full":
+            csa.csa2_quantize_append(self.shape, self.cache, b, 1, I["qpos"], I["kv"], I["idx_k"], I["swa_kv"],
+                                     ws=self.ws, stream=stream)
+        else:
+            csa.csa2_quantize_append(self.shape, self.cache, b, 1, I["qpos"], None, None, I["swa_kv"], ws=self.ws,
+                                     stream=stream)
+        hooks("append", 1)
+        idx = I.get("idx")
+        if wl.mode in ("full", "reindex"):
+            hooks("index", 0)
+            if wl.mode == "full":
+                csa.csa2_index_topk_full(self.shape, self.cache, b, 1, I["qpos"], I["idx_q"], wl.k, O["idx"],
+                                         wl.pool_blocks, O.get("pool"), O.get("pool_n"), max_ctx=self.max_ctx,
+                                         ws=self.ws, stream=stream)
+            else:
+                csa.csa2_index_topk_reindex(self.shape, self.cache, b, I["qpos"], I["idx_q"], I["pool"], I["pool_n"],
+                                            wl.k, O["idx"], ws=self.ws, stream=stream)
+            hooks("index", 1)
+            idx = O["idx"]
+        hooks("attend", 0)
+        csa.csa2_sparse_attend(self.shape, self.cache, b, 1, I["qpos"], I["q"], idx, wl.k, O["out"], ws=self.ws,
+                               stream=stream)
+        hooks("attend", 1)
+
+
+def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda") -> Step:
+    """Allocate and fill the cache of workload `name` (optionally a smaller batch, or the sequences
+    seq_offset .. seq_offset+batch-1 of it, as a data-parallel rank would) and its step inputs."""
+    wl = WORKLOADS[name]
+    B = wl.batch if batch is None else batch
+    seqs = torch.arange(seq_offset, seq_offset + B, device=device)
+    shape = csa.make_shape(wl.win)
+    N = wl.context
+    I, O = {}, {}
+    if wl.mode == "prefill":
+        p0 = N - wl.tq
+        cache = csa.Cache(B, N, 1 << (wl.tq + wl.win - 1).bit_length(), device=device)
+        _fill_range(cache, shape, wl.seed, seqs, 0, p0, device)
+        p = torch.arange(p0, N, device=device)
+        I["kv"] = _vals(wl.seed, "kv", seqs, p, 256)[0].contiguous()
+        I["idx_k"] = _vals(wl.seed, "ik", seqs, p, 256)[0].contiguous()
+        I["swa_kv"] = _vals(wl.seed, "swa", seqs, p, 256)[0].contiguous()
+        I["idx_q"] = _vals(wl.seed, "iq", seqs, p, 256)[0].contiguous()
+        I["q"] = _vals(wl.seed, "q", seqs, p, 2048)[0].reshape(wl.tq, 16, 128).contiguous()
+        O["idx"] = torch.empty(wl.tq, wl.k, dtype=torch.int32, device=device)
+        O["out"] = torch.empty(wl.tq, 16, 128, dtype=torch.bfloat16, device=device)
+        ws = csa.Workspace(shape, 1, wl.tq, wl.k, N)
+        return Step(wl, shape, cache, ws, I, O, 1, N)
+
+    qpos = torch.full((B,), N - 1, dtype=torch.int64, device=device)
+    I["qpos"] = qpos
+    qp = qpos.unsqueeze(1)
+    I["swa_kv"] = _vals(wl.seed, "swa", seqs, qp, 256)[:, 0].contiguous()
+    I["q"] = _vals(wl.seed, "q", seqs, qp, 2048)[:, 0].reshape(B, 16, 128).contiguous()
+    O["out"] = torch.empty(B, 16, 128, dtype=torch.bfloat16, device=device)
+    if wl.mode != "minimal":
+        I["idx_q"] = _vals(wl.seed, "iq", seqs, qp, 256)[:, 0].contiguous()
+        O["idx"] = torch.empty(B, wl.k, dtype=torch.int32, device=device)
+    if wl.mode == "full":
+        cache = csa.Cache(B, N, 128, device=device)
+        _fill_range(cache, shape, wl.seed, seqs, 0, N - 1, device)
+        I["kv"] = _vals(wl.seed, "kv", seqs, qp, 256)[:, 0].contiguous()
+        I["idx_k"] = _vals(wl.seed, "ik", seqs, qp, 256)[:, 0].contiguous()
+        if wl.pool_blocks:
+            O["pool"] = torch.empty(B, wl.pool_blocks, dtype=torch.int32, device=device)
+            O["pool_n"] = torch.empty(B, dtype=torch.int32, device=device)
+        ws = csa.Workspace(shape, B, 1, wl.k, N, wl.pool_blocks)
+    elif wl.mode == "reindex":
+        cache = csa.Cache(B, N, 128, device=device)
+        nblk = N // wl.bs
+        pool = distinct_sorted(wl.seed, "pool", seqs, nblk, wl.pool_blocks).to(torch.int32).contiguous()
+        I["pool"] = pool
+        I["pool_n"] = torch.full((B,), wl.pool_blocks, dtype=torch.int32, device=device)
+        _fill_blocks(cache, shape, wl.seed, seqs, pool, wl.bs, device)
+        _fill_window(cache, shape, wl.seed, seqs, N - wl.win, N - 1, device)
+        ws = csa.Workspace(shape, B, 1, wl.k, wl.pool_blocks * wl.bs)
+    else:  # minimal
+        cache = csa.Cache(B, N, 128, device=device, indexer=False)
+        idx = distinct_sorted(wl.seed, "sel", seqs, N - 1, wl.k).to(torch.int32).contiguous()
+        I["idx"] = idx
+        _fill_rows(cache, shape, wl.seed, seqs, idx, device)
+        _fill_window(cache, shape, wl.seed, seqs, N - wl.win, N - 1, device)
+        ws = csa.Workspace(shape, B, 1, wl.k, 8)
+    torch.cuda.synchronize()
+    return Step(wl, shape, cache, ws, I, O, B, N)
+
+
+def _fill_range(cache, shape, seed, seqs, p0, p1, device, chunk=2048):
+    B = seqs.numel()
+    for a in range(p0, p1, chunk):
+        t = min(chunk, p1 - a)
+        p = torch.arange(a, a + t, device=device)
+        pos = torch.full((B,), a, dtype=torch.int64, device=device)
+        kv = _vals(seed, "kv", seqs, p, 256).contiguous()
+        ik = _vals(seed, "ik", seqs, p, 256).contiguous() if cache.ik_data is not None else None
+        sw = _vals(seed, "swa", seqs, p, 256).contiguous()
+        csa.csa2_quantize_append(shape, cache, B, t, pos, kv, ik, sw)
+
+
+def _fill_window(cache, shape, seed, seqs, p0, p1, device):
+    B = seqs.numel()
+    p = torch.arange(p0, p1, device=device)
+    pos = torch.full((B,), p0, dtype=torch.int64, device=device)
+    sw = _vals(seed, "swa", seqs, p, 256).contiguous()
+    csa.csa2_quantize_append(shape, cache, B, p1 - p0, pos, None, None, sw)
+
+
+def _fill_blocks(cache, shape, seed, seqs, pool, bs, device, group=125):
+    B, P = pool.shape
+    off = torch.arange(bs, device=device)
+    for g0 in range(0, P, group):
+        g1 = min(P, g0 + group)
+        p = (pool[:, g0:g1].to(torch.int64).unsqueeze(-1) * bs + off).reshape(B, -1)
+        kv = _vals(seed, "kv", seqs, p, 256)
+        ik = _vals(seed, "ik", seqs, p, 256)
+        for j in range(g1 - g0):
+            pos = pool[:, g0 + j].to(torch.int64) * bs
+            csa.csa2_quantize_append(shape, cache, B, bs, pos, kv[:, j * bs:(j + 1) * bs].contiguous(),
+                                     ik[:, j * bs:(j + 1) * bs].contiguous(), None)
+
+
+def _fill_rows(cache, shape, seed, seqs, idx, device):
+    B, K = idx.shape
+    p = idx.to(torch.int64)
+    kv = _vals(seed, "kv", seqs, p, 256)
+    for j in range(K):
+        csa.csa2_quantize_append(shape, cache, B, 1, p[:, j].contiguous(), kv[:, j:j + 1].contiguous(), None, None)
