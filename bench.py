@@ -138,80 +138,29 @@ class Clocks:
 # ---------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------
-def oracle_sample(wl_name, budget_s=12.0, max_queries=None):
-    """Times the oracle on whole decode steps of sampled sequences of the workload; returns
-    (queries/s, description, threads)."""
-    import numpy as np
-    import torch
-
+def oracle_sample(wl_name, budget_s=12.0, context=None):
+    """Times the CPU oracle on whole decode steps of sampled sequences of the workload (their caches are
+    built first, untimed); returns (queries/s, description, threads)."""
     import oracle
-    import workloads as W
+    from oracle import workload as OW
 
-    wl = W.WORKLOADS[wl_name]
     oracle.build()
-    N = wl.context
+    wl = OW.workload(wl_name, context)
     seqs = [0, 1]
-    built = []
-    for b in seqs:
-        bt = torch.tensor([b])
-        c = oracle.SeqCache(cap=N, swa_cap=128)
-        if wl.mode == "reindex":
-            pool = W.distinct_sorted(wl.seed, "pool", bt, N // wl.bs, wl.pool_blocks)[0].to(torch.int32).numpy()
-            for g0 in range(0, wl.pool_blocks, 250):
-                blk = torch.from_numpy(pool[g0:g0 + 250].astype(np.int64))
-                p = (blk.unsqueeze(1) * wl.bs + torch.arange(wl.bs)).reshape(-1)
-                kv = W.cache_values(wl.seed, "kv", bt, p, 256)[0]
-                ik = W.cache_values(wl.seed, "ik", bt, p, 256)[0]
-                for j in range(blk.numel()):
-                    c.append(int(p[j * wl.bs]), kv=kv[j * wl.bs:(j + 1) * wl.bs], idx_k=ik[j * wl.bs:(j + 1) * wl.bs])
-        elif wl.mode == "full":
-            for a in range(0, N - 1, 8192):
-                p = torch.arange(a, min(N - 1, a + 8192))
-                c.append(a, kv=W.cache_values(wl.seed, "kv", bt, p, 256)[0], idx_k=W.cache_values(wl.seed, "ik", bt, p, 256)[0])
-            pool = None
-        else:
-            pool = None
-        pw = torch.arange(N - wl.win, N - 1)
-        c.append(N - wl.win, swa_kv=W.cache_values(wl.seed, "swa", bt, pw, 256)[0])
-        qp = torch.tensor([N - 1])
-        inp = {
-            "swa": W.cache_values(wl.seed, "swa", bt, qp, 256)[0],
-            "iq": W.cache_values(wl.seed, "iq", bt, qp, 256)[0, 0],
-            "q": W.cache_values(wl.seed, "q", bt, qp, 2048)[0, 0],
-            "kv": W.cache_values(wl.seed, "kv", bt, qp, 256)[0],
-            "ik": W.cache_values(wl.seed, "ik", bt, qp, 256)[0],
-        }
-        if wl.mode == "minimal":
-            inp["idx"] = W.distinct_sorted(wl.seed, "sel", bt, N - 1, wl.k)[0].to(torch.int32).numpy()
-            kvr = W.cache_values(wl.seed, "kv", bt, torch.from_numpy(inp["idx"].astype(np.int64)), 256)[0]
-            for j, pp in enumerate(inp["idx"]):
-                c.append(int(pp), kv=kvr[j:j + 1])
-        built.append((c, pool, inp))
-
-    def step(c, pool, inp):
-        if wl.mode == "reindex":
-            c.append(N - 1, swa_kv=inp["swa"])
-            idx = c.index_topk_reindex(N - 1, inp["iq"], pool, len(pool), k=wl.k)
-        elif wl.mode == "full":
-            c.append(N - 1, kv=inp["kv"], idx_k=inp["ik"], swa_kv=inp["swa"])
-            r = c.index_topk_full(N - 1, inp["iq"], k=wl.k, pool_blocks=wl.pool_blocks)
-            idx = r[0] if wl.pool_blocks else r
-        else:
-            c.append(N - 1, swa_kv=inp["swa"])
-            idx = inp["idx"]
-        return c.sparse_attend(N - 1, inp["q"], idx)
-
+    built = [OW.build_sequence(wl, b) for b in seqs]
+    rows = [0] if wl.mode == "prefill" else None
     n = 0
     t0 = time.perf_counter()
     while True:
-        for c, pool, inp in built:
-            step(c, pool, inp)
+        for c, inp in built:
+            OW.run_step(c, wl, inp, rows=rows)
             n += 1
         el = time.perf_counter() - t0
-        if el >= budget_s or (max_queries and n >= max_queries):
+        if el >= budget_s:
             break
-    desc = (f"{n} whole decode steps of {wl_name} (sequences {seqs} repeated, cache already resident in host "
-            f"memory), single-threaded C oracle, fp64, {el:.1f} s")
+    what = "prefill query rows (one row per step)" if wl.mode == "prefill" else "whole decode steps"
+    desc = (f"{n} {what} of {wl_name} (sequences {seqs} repeated, cache resident in host memory), "
+            f"single-threaded C oracle, fp64, {el:.1f} s")
     return n / el, desc, 1
 
 
@@ -234,7 +183,8 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     wl = W.WORKLOADS[args.workload]
     B = args.batch or wl.batch
-    step = G.build(args.workload, batch=B, seq_offset=rank * B)
+    step = G.build(args.workload, batch=B, seq_offset=rank * B, context=args.context or None)
+    wl = step.wl
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -316,7 +266,7 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic (seeded near-Gaussian bf16, sigma 1, clipped to +-26)",
-        "config": {"workload": args.workload, "mode": wl.mode, "batch_per_gpu": B, "context": wl.context,
+        "config": {"workload": args.workload + (f"@ctx{wl.context}" if args.context else ""), "mode": wl.mode, "batch_per_gpu": B, "context": wl.context,
                    "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": 16, "head_dim": 128,
                    "indexer": "4 heads x 64, FP4", "kv_cache": "E2M1 + E4M3/16 (FP4), window FP8",
                    "window": wl.win, "parallelism": f"dp{world}",
@@ -330,7 +280,7 @@ def run_gpu(args):
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
-        v, desc, cores = oracle_sample(args.workload, budget_s=args.cpu_budget)
+        v, desc, cores = oracle_sample(args.workload, budget_s=args.cpu_budget, context=args.context or None)
         line["cpu_baseline"] = {"value": round(v, 3), "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
     print(json.dumps(line), flush=True)
 
@@ -388,7 +338,7 @@ def run_reference(args):
     if rank != 0:
         return
     per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
-    v, desc, cores = oracle_sample(args.workload, budget_s=per_step * max(1, args.steps))
+    v, desc, cores = oracle_sample(args.workload, budget_s=per_step * max(1, args.steps), context=args.context or None)
     line = {"metric": METRIC, "value": round(v, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
@@ -405,6 +355,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--batch", type=int, default=0, help="sequences per GPU (default: the workload's)")
+    ap.add_argument("--context", type=int, default=0, help="context override (profiling small cases)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)

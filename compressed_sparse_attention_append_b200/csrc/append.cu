@@ -105,6 +105,9 @@ __global__ void __launch_bounds__(192) append_kernel(AppendArgs a) {
             if (task == 32 && i == 0) set_status(a.status, CSA2_DEV_BAD_POS);
             return;
         }
+        // the ring keeps the latest swa_cap positions: older tokens of this call would share a
+        // slot with a newer one, so they are not written
+        if ((int64_t)i < (int64_t)a.t - a.c.swa_cap) return;
         const int g = task - 32;
         float x[16];
         load16_bf16(a.swa_kv + tok * 256 + g * 16, x);

@@ -1,0 +1,69 @@
+"""The five workloads at full size, in the launch configuration bench.py times, checked on sampled
+sequences (prefill: sampled query rows) against the oracle: index sets and pools identical, attention
+within tolerance."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import workload as OW
+from workloads import gpu as G
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("full_b1_n4096", [0]),
+    ("full_b64_n131072", [0, 63]),
+    ("reindex_b128_n1m", [0, 77, 127]),
+    ("minimal_b256_n262144", [0, 100, 255]),
+]
+
+
+def _cmp_attn(out, of, ro, tol=2e-3):
+    assert torch.equal(out, of.to(torch.bfloat16))
+    err = np.abs(of.double().cpu().numpy() - ro).max()
+    assert err <= tol, err
+
+
+@pytest.mark.parametrize("name,seqs", CASES)
+def test_decode_workload_sampled(orc, name, seqs):
+    step = G.build(name)
+    of = torch.empty(step.batch, 16, 128, dtype=torch.float32, device="cuda")
+    step.run(out_f32=of)
+    import compressed_sparse_attention_append_b200 as csa
+
+    assert csa.csa2_get_device_status(step.ws) == 0
+    wl = step.wl
+    for b in seqs:
+        c, inp = OW.build_sequence(wl, b)
+        r = OW.run_step(c, wl, inp)
+        if wl.mode != "minimal":
+            assert np.array_equal(step.outputs["idx"][b].cpu().numpy(), r["idx"]), b
+        if wl.mode == "full" and wl.pool_blocks:
+            assert np.array_equal(step.outputs["pool"][b].cpu().numpy(), r["pool"])
+            assert int(step.outputs["pool_n"][b]) == r["pool_n"]
+        _cmp_attn(step.outputs["out"][b], of[b], r["out"])
+    # a second step on the same state gives the same result (counters cleared, appends idempotent)
+    prev = {k: v.clone() for k, v in step.outputs.items()}
+    step.run()
+    for k, v in step.outputs.items():
+        assert torch.equal(v, prev[k]), k
+    del step
+    torch.cuda.empty_cache()
+
+
+def test_prefill_workload_sampled_rows(orc):
+    name = "prefill_t4096_at_1m"
+    step = G.build(name)
+    wl = step.wl
+    of = torch.empty(wl.tq, 16, 128, dtype=torch.float32, device="cuda")
+    step.run(out_f32=of)
+    torch.cuda.synchronize()
+    rows = [0, 1, 2047, 4095]
+    c, inp = OW.build_sequence(wl, 0)
+    r = OW.run_step(c, wl, inp, rows=rows)
+    for i in rows:
+        idx, ro, _ = r["rows"][i]
+        assert np.array_equal(step.outputs["idx"][i].cpu().numpy(), idx), i
+        _cmp_attn(step.outputs["out"][i], of[i], ro)
+    del step
+    torch.cuda.empty_cache()

@@ -83,10 +83,13 @@ class Step:
         hooks("attend", 1)
 
 
-def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda") -> Step:
+def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda", context=None) -> Step:
     """Allocate and fill the cache of workload `name` (optionally a smaller batch, or the sequences
-    seq_offset .. seq_offset+batch-1 of it, as a data-parallel rank would) and its step inputs."""
+    seq_offset .. seq_offset+batch-1 of it, as a data-parallel rank would; optionally another context
+    length, for profiling small cases) and its step inputs."""
     wl = WORKLOADS[name]
+    if context:
+        wl = dataclasses.replace(wl, context=context)
     B = wl.batch if batch is None else batch
     seqs = torch.arange(seq_offset, seq_offset + B, device=device)
     shape = csa.make_shape(wl.win)
