@@ -22,7 +22,7 @@ csa2_status check_shape(const csa2_shape* s) {
 // planes: 1 = main, 2 = indexer, 4 = window
 csa2_status check_cache(const csa2_cache* c, int planes) {
     if (!c || c->cap <= 0 || c->swa_cap <= 0 || (c->swa_cap & (c->swa_cap - 1))) return CSA2_ERR_INVALID_ARG;
-    if (c->cap > (int64_t)0x7FFFFFFF) return CSA2_ERR_CAPACITY;  // positions are stored as int32
+    if (c->cap > ((int64_t)1 << 30)) return CSA2_ERR_CAPACITY;  // positions travel as int32 with headroom
     if (planes & 1) {
         if (!c->kv_data || !c->kv_scale || !al16(c->kv_data) || !al16(c->kv_scale)) return CSA2_ERR_INVALID_ARG;
     }

@@ -152,7 +152,7 @@ inline IndexPlan make_index_plan(int rows, int k, int64_t max_scan, int pool_blo
     p.pool_blocks = pool_blocks;
     p.units_max = (int)((max_scan + kBS - 1) / kBS);
     if (p.units_max < 1) p.units_max = 1;
-    const int items_target = 148 * 8;
+    const int items_target = 148 * 4;
     int chunks_target = (items_target + rows - 1) / rows;
     if (chunks_target < 1) chunks_target = 1;
     int cu = (p.units_max + chunks_target - 1) / chunks_target;
@@ -166,14 +166,17 @@ inline IndexPlan make_index_plan(int rows, int k, int64_t max_scan, int pool_blo
 }
 
 inline AttendPlan make_attend_plan(int rows, int k, int win) {
+    // CTAs of 8 warps, two per SM: about 296 CTAs in flight; a split covers at least 256 keys
+    // (two 16-key tiles per warp) so that each warp keeps tiles in flight
     AttendPlan a{};
     a.rows = rows;
     a.nk_max = k + win;
-    int tiles = (a.nk_max + 63) / 64;
-    int splits = (2 * 148 + rows - 1) / rows;
+    const int units = (a.nk_max + 127) / 128;  // 128 keys = one tile per warp
+    int max_splits = units / 2 > 1 ? units / 2 : 1;
+    int splits = 296 / (rows > 0 ? rows : 1);
     if (splits < 1) splits = 1;
-    if (splits > tiles) splits = tiles;
-    a.kps = ((tiles + splits - 1) / splits) * 64;
+    if (splits > max_splits) splits = max_splits;
+    a.kps = ((units + splits - 1) / splits) * 128;
     a.splits = (a.nk_max + a.kps - 1) / a.kps;
     return a;
 }

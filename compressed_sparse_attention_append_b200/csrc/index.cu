@@ -8,21 +8,28 @@
 // to 2,048) form the pool. sec. XI: indexer queries and keys are FP4.
 //
 // Score (this build's reading; the pages give no formula): score(p) = sum_h q_h . k_{p,h} over 4
-// heads x 64 channels of dequantised FP4 values. The score is EXACT: per 16-channel block, the
-// sum of 16 products of E2M1 values is accumulated in fp16 in two halves of 8 products (each a
-// multiple of 1/4 below 288, exact in fp16), the two halves are added in fp32 (exact, < 576),
-// multiplied by the fp32 product of the two E4M3 scales (exact, <= 8 significant bits; the
-// product has <= 20 bits), and the 16 block partials are summed in fp64 (all terms are multiples
-// of 2^-20 below 2^31). Ranking is by score descending, ties to the lower position (to the lower
-// block id for the pool), so the selected set is unique.
+// heads x 64 channels of dequantised FP4 values, computed EXACTLY as the integer S = score * 2^20:
+//   * an E2M1 code c decodes to the integer 2*value(c) in {0, +-1, +-2, +-3, +-4, +-6, +-8, +-12}
+//     through a byte permute (prmt) of the table {0,1,2,3,4,6,8,12}: the permute's sign-replicate
+//     mode turns the codes of one sign into 0, so one prmt of the codes gives the magnitudes of
+//     the positive channels and one prmt of the sign-flipped codes those of the negative ones;
+//   * a 16-channel block's dot product D = sum (2q)(2k) comes from dp4a (|D| <= 2304);
+//   * an E4M3 scale s = M * 2^(E-10) (M <= 15, E >= 1) enters as the integer f(s) = M * 2^(E-1)
+//     (<= 245760); D * f(s_k) fits in int32 and (D * f(s_k)) * f(s_q) is added to an int64
+//     with one wide multiply-add (each term < 2^47, the sum of 16 terms < 2^51).
+// No floating-point conversion runs in the scoring loop. Ranking is by S descending, ties to the
+// lower position (to the lower block id for the pool); S is the same integer the exact rational
+// score gives, so the selected set is unique and reproducible.
 //
 // Structure (one kernel, persistent CTAs taking work items from an atomic counter):
-//   item = (query row, chunk of 8-position units). A CTA scores the chunk two units per warp
-//   step (16 positions, 2 KB of indexer keys, loaded as coalesced 16-byte vectors), keeps a
-//   running local Top-k in shared memory (admission threshold + radix select), and emits its
-//   local Top-k to the row's candidate list in the workspace. The CTA that finishes a row's
-//   last chunk merges the candidates (and, for the pool, the per-unit block maxima) into the
-//   final ascending outputs and clears the row's counters.
+//   item = (chunk of 8-position units, query row), chunk-major so that later chunks of a row start
+//   with the admission threshold left by its earlier chunks. Each warp scores two units per step
+//   (16 positions, 2 KB of keys + 256 B of scales) from a private 3-stage cp.async ring; a running
+//   local Top-k sits in shared memory (admission threshold + radix select over orderable keys,
+//   skipping the bits all keys share and histogramming with match_any). A CTA emits its local
+//   Top-k to the row's candidate list; the CTA that finishes a row's last chunk merges the
+//   candidates (and, for the pool, the per-unit block maxima) into the final ascending outputs
+//   and clears the row's counters.
 #include "csa2_internal.cuh"
 
 namespace csa2 {
@@ -31,30 +38,64 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSubUnits = 256;            // units scored between two selection flushes
-constexpr int kNewCap = kSubUnits * kBS;  // admissions per sub-chunk, worst case
+constexpr int kStages = 2;
+constexpr int kUnitsPerStep = 4;                      // units scored by one warp step (32 positions)
+constexpr int kStepBytes = kUnitsPerStep * (1024 + 128);  // codes + scales of 4 units
+constexpr int kStagingBytes = kWarps * kStages * kStepBytes;
+constexpr int kStepsPerFlush = 4;                     // warp steps between two selection flushes
+constexpr int kSubUnits = kWarps * kUnitsPerStep * kStepsPerFlush;  // 128 units
+constexpr int kNewCap = kSubUnits * kBS;              // admissions per sub-chunk, worst case
 
-struct Smem {
+struct SelBuf {
     unsigned long long* keep_key[2];
     int* keep_pos[2];
     unsigned long long* new_key;
     int* new_pos;
-    unsigned int* hist;      // 256
-    int kcap;
 };
 
-struct __align__(16) SmemScalars {
+struct __align__(16) Scal {
     int cur, nkeep, nnew, digit, above, cnt, last, misc;
-    unsigned long long thr, prefix;
-    float qscale[16];
-    __align__(16) uint8_t qcode[128];  // read back as 16-byte vectors
+    unsigned long long thr, prefix, red_and[kWarps], red_or[kWarps];
+    int qf[16];
+    __align__(16) uint8_t qcode[128];
+    __align__(16) uint32_t qv[128];   // [chunk s][word i][pa, pb, na, nb]
 };
+
+// ---- integer decode of E2M1 codes -------------------------------------------------------------
+// prmt with the table bytes {0,1,2,3,4,6,8,12}: selector nibble = code; a set sign bit selects the
+// sign-replicate mode, whose result is 0 because every table byte is positive.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+constexpr uint32_t kTab0 = 0x03020100u, kTab1 = 0x0C080604u;
+
+// sum over the 8 channels of word w of (2q)(2k); qa/qb = 2q of channels 0..3 / 4..7 as int8x4
+__device__ __forceinline__ int dot8(uint32_t w, uint32_t qa, uint32_t qb, uint32_t nqa, uint32_t nqb, int acc) {
+    const uint32_t wx = w ^ 0x88888888u;
+    acc = __dp4a((int)prmt(kTab0, kTab1, w), (int)qa, acc);
+    acc = __dp4a((int)prmt(kTab0, kTab1, wx), (int)nqa, acc);
+    acc = __dp4a((int)prmt(kTab0, kTab1, w >> 16), (int)qb, acc);
+    acc = __dp4a((int)prmt(kTab0, kTab1, wx >> 16), (int)nqb, acc);
+    return acc;
+}
+
+// f(s) = M * 2^(E-1) for an E4M3 byte (value M * 2^(E-10)); sign applied; NaN codes give 0.
+__device__ __forceinline__ int e4m3_fixed(int byte) {
+    const int e = (byte >> 3) & 15, m = byte & 7;
+    if (e == 15 && m == 7) return 0;
+    const int M = e ? (8 | m) : m;
+    const int v = M << (e ? e - 1 : 0);
+    return (byte & 0x80) ? -v : v;
+}
 
 __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
     return __shfl_xor_sync(0xffffffffu, v, m);
 }
+__device__ __forceinline__ long long shfl_xor_s64(long long v, int m) { return __shfl_xor_sync(0xffffffffu, v, m); }
 
-// ---- query quantisation (same codec as the cache) ------------------------------------------
+// ---- query quantisation (same codec as the cache), 8 threads per 16-channel block ---------------
 __device__ __forceinline__ uint32_t q_f32x2_to_e2m1x2(float lo, float hi) {
     uint16_t r;
     asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tmov.b16 %0, {t, 0};\n\t}"
@@ -67,59 +108,82 @@ __device__ __forceinline__ uint32_t q_f32_to_e4m3(float v) {
     return r & 0xFF;
 }
 
-__device__ void quantize_query(const uint16_t* q, SmemScalars& S) {
+__device__ void quantize_query(const uint16_t* q, Scal& S, const int* kf_lut) {
     const int t = threadIdx.x;
-    if (t < 16) {
-        float x[16];
-        const uint4 a = *reinterpret_cast<const uint4*>(q + t * 16);
-        const uint4 b = *reinterpret_cast<const uint4*>(q + t * 16 + 8);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            x[2 * i] = __uint_as_float(w[i] << 16);
-            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-            amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
-        }
+    if (t < 128) {
+        const int blk = t >> 3, sub = t & 7;  // 2 channels per thread
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(q + blk * 16 + 2 * sub);
+        const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xFFFF0000u);
+        float amax = fmaxf(fabsf(x0), fabsf(x1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
         const uint32_t sc = q_f32_to_e4m3(__fdiv_rn(amax, 6.0f));
-        const float s = e4m3_to_f32((uint8_t)sc);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            S.qcode[t * 8 + j] = (s == 0.f) ? 0 : (uint8_t)q_f32x2_to_e2m1x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
-        S.qscale[t] = s;
+        const float s = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)sc, __NV_E4M3)));
+        S.qcode[blk * 8 + sub] = (s == 0.f) ? 0 : (uint8_t)q_f32x2_to_e2m1x2(__fdiv_rn(x0, s), __fdiv_rn(x1, s));
+        if (sub == 0) S.qf[blk] = kf_lut[sc];
     }
 }
 
+// 2 * value of an E2M1 code as a signed byte
+__device__ __forceinline__ uint32_t e2m1_int2(uint32_t c) {
+    const uint32_t mag = (prmt(kTab0, kTab1, c & 7) & 0xFF);
+    return (c & 8) ? ((0u - mag) & 0xFF) : mag;
+}
+
 // ---- CTA radix select ----------------------------------------------------------------------------
-// Elements i < na come from (ka, pa), the rest from (kb, pb). Writes the top `K` (key desc,
-// pos asc) into (ko, po) in arbitrary order; returns through S.thr a lower bound of the kept keys.
+// Elements i < na: (ka, pa); the rest: (kb, pb). Writes the top K (key desc, pos asc) into (ko, po);
+// S.thr becomes a lower bound of the kept keys.
 __device__ void cta_select(const unsigned long long* ka, const int* pa, int na, const unsigned long long* kb,
-                           const int* pb, int nb, int K, unsigned long long* ko, int* po, Smem& M, SmemScalars& S) {
+                           const int* pb, int nb, int K, unsigned long long* ko, int* po, unsigned int* hist,
+                           Scal& S) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = na + nb;
     auto key_at = [&](int i) { return i < na ? ka[i] : kb[i - na]; };
     auto pos_at = [&](int i) { return i < na ? pa[i] : pb[i - na]; };
-
-    unsigned long long prefix = 0, mask = 0;
+    // bits shared by every key are skipped
+    unsigned long long va = ~0ull, vo = 0ull;
+    for (int i = tid; i < n; i += kThreads) { const unsigned long long k = key_at(i); va &= k; vo |= k; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) { va &= shfl_xor_u64(va, o); vo |= shfl_xor_u64(vo, o); }
+    if (lane == 0) { S.red_and[warp] = va; S.red_or[warp] = vo; }
+    __syncthreads();
+    va = ~0ull; vo = 0ull;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) { va &= S.red_and[w]; vo |= S.red_or[w]; }
+    const unsigned long long diff = va ^ vo;
+    int top = diff ? 63 - __clzll((long long)diff) : -1;
+    unsigned long long mask = (top >= 63) ? 0ull : ~((2ull << top) - 1ull);
+    unsigned long long prefix = va & mask;
+    if (top < 0) { mask = ~0ull; prefix = va; }
     int kr = K;
     bool exact = false;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        M.hist[tid] = 0;  // kThreads == 256 bins
+    while (top >= 0) {
+        const int shift = top >= 7 ? top - 7 : 0;
+        const int nbits = top - shift + 1;
+        const unsigned int dmask = (1u << nbits) - 1u;
+        hist[tid] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += kThreads) {
-            const unsigned long long key = key_at(i);
-            if ((key & mask) == prefix) atomicAdd(&M.hist[(key >> shift) & 255], 1u);
+        for (int base = 0; base < n; base += kThreads) {
+            const int i = base + tid;
+            int d = -1;
+            if (i < n) {
+                const unsigned long long key = key_at(i);
+                if ((key & mask) == prefix) d = (int)((key >> shift) & dmask);
+            }
+            const unsigned int peers = __match_any_sync(0xffffffffu, d);
+            if (d >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
         }
         __syncthreads();
         if (warp == 0) {
             // lane L owns bins 255-8L ... 248-8L (descending)
             unsigned int c[8], sum = 0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) { c[j] = M.hist[255 - 8 * lane - j]; sum += c[j]; }
+            for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * lane - j]; sum += c[j]; }
             unsigned int incl = sum;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
+                const unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
                 if (lane >= o) incl += v;
             }
             const unsigned int excl = incl - sum;
@@ -140,33 +204,39 @@ __device__ void cta_select(const unsigned long long* ka, const int* pa, int na, 
         __syncthreads();
         kr -= S.above;
         prefix |= (unsigned long long)S.digit << shift;
-        mask |= 0xFFull << shift;
-        if (S.cnt == kr) { exact = true; }
+        mask |= (unsigned long long)dmask << shift;
+        exact = (S.cnt == kr);
+        top = shift - 1;
         __syncthreads();
         if (exact) break;
     }
-    // tie on the full key: the kr lowest positions among key == prefix
+    // all keys equal down to the last bit: the kr lowest positions among key == prefix
     unsigned int pthr = 0xFFFFFFFFu;
     if (!exact) {
         unsigned int pp = 0, pm = 0;
         int r = kr;
         for (int shift = 24; shift >= 0; shift -= 8) {
-            M.hist[tid] = 0;
+            hist[tid] = 0;
             __syncthreads();
-            for (int i = tid; i < n; i += kThreads) {
-                if (key_at(i) != prefix) continue;
-                const unsigned int p = (unsigned int)pos_at(i);
-                if ((p & pm) == pp) atomicAdd(&M.hist[(p >> shift) & 255], 1u);
+            for (int base = 0; base < n; base += kThreads) {
+                const int i = base + tid;
+                int d = -1;
+                if (i < n && key_at(i) == prefix) {
+                    const unsigned int p = (unsigned int)pos_at(i);
+                    if ((p & pm) == pp) d = (int)((p >> shift) & 255u);
+                }
+                const unsigned int peers = __match_any_sync(0xffffffffu, d);
+                if (d >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
             }
             __syncthreads();
             if (warp == 0) {
                 unsigned int c[8], sum = 0;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) { c[j] = M.hist[8 * lane + j]; sum += c[j]; }
+                for (int j = 0; j < 8; ++j) { c[j] = hist[8 * lane + j]; sum += c[j]; }
                 unsigned int incl = sum;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
-                    unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    const unsigned int v = __shfl_up_sync(0xffffffffu, incl, o);
                     if (lane >= o) incl += v;
                 }
                 const unsigned int excl = incl - sum;
@@ -187,9 +257,8 @@ __device__ void cta_select(const unsigned long long* ka, const int* pa, int na, 
             __syncthreads();
             if (done) break;
         }
-        pthr = pp | ~pm;  // every position with the chosen prefix qualifies
+        pthr = pp | ~pm;
     }
-    // compaction
     if (tid == 0) S.misc = 0;
     __syncthreads();
     for (int base = 0; base < n; base += kThreads) {
@@ -200,8 +269,7 @@ __device__ void cta_select(const unsigned long long* ka, const int* pa, int na, 
         if (i < n) {
             key = key_at(i);
             p = pos_at(i);
-            if (exact) sel = (key & mask) >= prefix;
-            else sel = key > prefix || (key == prefix && (unsigned int)p <= pthr);
+            sel = exact ? (key & mask) >= prefix : (key > prefix || (key == prefix && (unsigned int)p <= pthr));
         }
         const unsigned int bal = __ballot_sync(0xffffffffu, sel);
         int wbase = 0;
@@ -214,32 +282,30 @@ __device__ void cta_select(const unsigned long long* ka, const int* pa, int na, 
         }
     }
     __syncthreads();
-    if (tid == 0) S.thr = prefix;
+    if (tid == 0 && prefix > S.thr) S.thr = prefix;
     __syncthreads();
 }
 
-// Merge the pending admissions into the running Top-K.
-__device__ void flush(Smem& M, SmemScalars& S, int K) {
+__device__ void flush(SelBuf& B, unsigned int* hist, Scal& S, int K) {
     const int nk = S.nkeep, nn = S.nnew, cur = S.cur;
     if (nn == 0) return;
     if (nk + nn <= K) {
         for (int i = threadIdx.x; i < nn; i += kThreads) {
-            M.keep_key[cur][nk + i] = M.new_key[i];
-            M.keep_pos[cur][nk + i] = M.new_pos[i];
+            B.keep_key[cur][nk + i] = B.new_key[i];
+            B.keep_pos[cur][nk + i] = B.new_pos[i];
         }
         __syncthreads();
         if (threadIdx.x == 0) { S.nkeep = nk + nn; S.nnew = 0; }
         __syncthreads();
         return;
     }
-    cta_select(M.keep_key[cur], M.keep_pos[cur], nk, M.new_key, M.new_pos, nn, K, M.keep_key[cur ^ 1],
-               M.keep_pos[cur ^ 1], M, S);
+    cta_select(B.keep_key[cur], B.keep_pos[cur], nk, B.new_key, B.new_pos, nn, K, B.keep_key[cur ^ 1],
+               B.keep_pos[cur ^ 1], hist, S);
     if (threadIdx.x == 0) { S.cur = cur ^ 1; S.nkeep = K; S.nnew = 0; }
     __syncthreads();
 }
 
-// Admit (key, pos) from lanes with `valid`, warp-aggregated.
-__device__ __forceinline__ void admit(Smem& M, SmemScalars& S, bool valid, unsigned long long key, int pos) {
+__device__ __forceinline__ void admit(SelBuf& B, Scal& S, bool valid, unsigned long long key, int pos) {
     const int lane = threadIdx.x & 31;
     const unsigned int bal = __ballot_sync(0xffffffffu, valid);
     if (!bal) return;
@@ -248,12 +314,12 @@ __device__ __forceinline__ void admit(Smem& M, SmemScalars& S, bool valid, unsig
     base = __shfl_sync(0xffffffffu, base, 0);
     if (valid) {
         const int o = base + __popc(bal & ((1u << lane) - 1));
-        M.new_key[o] = key;
-        M.new_pos[o] = pos;
+        B.new_key[o] = key;
+        B.new_pos[o] = pos;
     }
 }
 
-// Ascending bitonic sort of n <= kNewCap int32 values in `a` (padded with INT_MAX to a power of 2).
+// Ascending bitonic sort of n int32 values in `a` (room for the next power of two of n).
 __device__ void sort_ascending(int* a, int n) {
     int P = 1;
     while (P < n) P <<= 1;
@@ -301,111 +367,120 @@ __device__ RowInfo row_info(const IndexArgs& a, int row) {
     return r;
 }
 
-// ---- scoring of two 8-position units by one warp --------------------------------------------------
+// Block id of unit u of row R and its number of scoreable positions (0..8); -1 / 0 when the unit is
+// past the chunk or its pool id is invalid.
+__device__ __forceinline__ void unit_info(const IndexArgs& a, const RowInfo& R, int u, int u_end, int& blk, int& nv,
+                                          uint32_t* status) {
+    blk = -1;
+    nv = 0;
+    if (u >= u_end) return;
+    int id = u;
+    if (a.reindex) {
+        id = __ldg(a.pool + (size_t)R.b * a.pool_stride + u);
+        if (id < 0 || (int64_t)id * kBS >= a.c.cap) {
+            set_status(status, CSA2_DEV_BAD_POOL);
+            return;
+        }
+    }
+    const int64_t p0 = (int64_t)id * kBS;
+    int64_t n = R.qpos - p0 + 1;
+    if (a.c.cap - p0 < n) n = a.c.cap - p0;
+    if (n <= 0) return;
+    blk = id;
+    nv = n > kBS ? kBS : (int)n;
+}
+
+// One warp step: units u .. u+3. Lane u (< 4) resolves unit u; the result is broadcast.
+// Staging: codes of unit j at 1024*j, scales at 4096 + 128*j.
+__device__ __forceinline__ int stage_step(const IndexArgs& a, const RowInfo& R, int ustep, int u_end,
+                                          unsigned char* st, uint32_t* status) {
+    const int lane = threadIdx.x & 31;
+    int blk = -1, nv = 0;
+    if (lane < kUnitsPerStep) unit_info(a, R, ustep + lane, u_end, blk, nv, status);
+    const int packed = (blk << 4) | nv;  // blk < 2^26 (cap <= 2^30 positions); -1 packs to -16
+    const uint8_t* base = a.c.ik_data + (size_t)R.b * a.c.cap * kIKBytes;
+    const uint8_t* sbase = a.c.ik_scale + (size_t)R.b * a.c.cap * kIKScales;
+#pragma unroll
+    for (int u = 0; u < kUnitsPerStep; ++u) {
+        const int pk = __shfl_sync(0xffffffffu, packed, u);
+        const int b = pk >> 4, n = pk & 15;
+        if (b < 0) continue;
+        const size_t row0 = (size_t)b * kBS;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int off = 512 * h + 16 * lane;  // position 4h + lane/8 of the unit
+            if (4 * h + (lane >> 3) < n) cp_async16(st + 1024 * u + off, base + row0 * kIKBytes + off);
+        }
+        if ((lane >> 3) == u && (lane & 7) < n)
+            cp_async16(st + 4096 + 128 * u + 16 * (lane & 7), sbase + (row0 + (lane & 7)) * kIKScales);
+    }
+    return packed;
+}
+
+// Scores the staged step (lane (m, s), load j: position (j&1)*4+m of unit j>>1, channels 32s..32s+31),
+// reduce-scatters over the octet so that lane (m, s) holds the score of position (s&1)*4+m of unit s>>1.
 template <bool RELU>
-__device__ __forceinline__ void score_pair(const IndexArgs& a, const RowInfo& R, int unitA, int u_end,
-                                           const uint32_t (&qh)[16], float qs0, float qs1, Smem& M,
-                                           SmemScalars& S, unsigned long long thr, unsigned long long* bmax_row,
-                                           uint32_t* status) {
+__device__ __forceinline__ void score_step(const unsigned char* st, int packed, int ustep, const uint32_t (&qv)[16],
+                                           int qf0, int qf1, const int* kf_lut, SelBuf& B, Scal& S,
+                                           unsigned long long thr, unsigned long long* bmax_row) {
     const int lane = threadIdx.x & 31;
     const int m = lane >> 3, s = lane & 7;
-    int blk[2];
-    bool uvalid[2];
+    long long v[8];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-        const int unit = unitA + u;
-        uvalid[u] = unit < u_end;
-        blk[u] = unit;
-        if (uvalid[u] && a.reindex) {
-            const int id = a.pool[(size_t)R.b * a.pool_stride + unit];
-            if (id < 0 || (int64_t)id * kBS >= a.c.cap) {
-                if (lane == 0) set_status(status, CSA2_DEV_BAD_POOL);
-                uvalid[u] = false;
-            }
-            blk[u] = id;
+    for (int j = 0; j < 8; ++j) {
+        const uint4 w = *reinterpret_cast<const uint4*>(st + 1024 * (j >> 1) + 512 * (j & 1) + 16 * lane);
+        const uint32_t sc = *reinterpret_cast<const uint16_t*>(st + 4096 + 128 * (j >> 1) + 16 * ((j & 1) * 4 + m) + 2 * s);
+        int d0 = dot8(w.x, qv[0], qv[1], qv[2], qv[3], 0);
+        d0 = dot8(w.y, qv[4], qv[5], qv[6], qv[7], d0);
+        int d1 = dot8(w.z, qv[8], qv[9], qv[10], qv[11], 0);
+        d1 = dot8(w.w, qv[12], qv[13], qv[14], qv[15], d1);
+        v[j] = (long long)(d0 * kf_lut[sc & 0xFF]) * qf0 + (long long)(d1 * kf_lut[sc >> 8]) * qf1;
+    }
+    if (RELU) {  // head s>>1 lives on lanes s and s^1
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            v[j] += shfl_xor_s64(v[j], 1);
+            v[j] = (v[j] > 0 && (s & 1) == 0) ? v[j] : 0;
         }
     }
-    // loads: j -> unit j>>1, unit position (j&1)*4 + m, channel chunk s (32 channels)
-    uint4 w[4];
-    uint32_t sc[4];
-    bool pv[4];
+    // reduce-scatter over the octet: lane s ends with position j = s
+    const bool b2 = s & 4, b1 = s & 2, b0 = s & 1;
+    long long w4[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int u = j >> 1;
-        const int64_t p = (int64_t)blk[u] * kBS + (j & 1) * 4 + m;
-        pv[j] = uvalid[u] && p <= R.qpos && p < a.c.cap;
-        w[j] = make_uint4(0, 0, 0, 0);
-        sc[j] = 0;
-        if (pv[j]) {
-            const size_t row = (size_t)R.b * a.c.cap + (size_t)p;
-            w[j] = __ldg(reinterpret_cast<const uint4*>(a.c.ik_data + row * kIKBytes) + s);
-            sc[j] = __ldg(reinterpret_cast<const uint16_t*>(a.c.ik_scale + row * kIKScales) + s);
-        }
+    for (int i = 0; i < 4; ++i) {
+        const long long keep = b2 ? v[4 + i] : v[i], send = b2 ? v[i] : v[4 + i];
+        w4[i] = keep + shfl_xor_s64(send, 4);
     }
-    double v[4];
+    long long w2[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t k0[4], k1[4], k2[4], k3[4];
-        e2m1x8_to_h2x4(w[j].x, k0);
-        e2m1x8_to_h2x4(w[j].y, k1);
-        e2m1x8_to_h2x4(w[j].z, k2);
-        e2m1x8_to_h2x4(w[j].w, k3);
-        uint32_t acc0 = 0, acc1 = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc0 = hfma2(qh[i], k0[i], acc0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc0 = hfma2(qh[4 + i], k1[i], acc0);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc1 = hfma2(qh[8 + i], k2[i], acc1);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc1 = hfma2(qh[12 + i], k3[i], acc1);
-        const float2 ks = h2_to_f2(e4m3x2_to_h2((uint16_t)sc[j]));
-        const float2 f0 = h2_to_f2(acc0), f1 = h2_to_f2(acc1);
-        const float p0 = (f0.x + f0.y) * (qs0 * ks.x);
-        const float p1 = (f1.x + f1.y) * (qs1 * ks.y);
-        v[j] = (double)p0 + (double)p1;
+    for (int i = 0; i < 2; ++i) {
+        const long long keep = b1 ? w4[2 + i] : w4[i], send = b1 ? w4[i] : w4[2 + i];
+        w2[i] = keep + shfl_xor_s64(send, 2);
     }
-    if (RELU) {
-        // head h = s >> 1 lives on lanes s and s^1: complete each head's dot first
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[j] += __shfl_xor_sync(0xffffffffu, v[j], 1);
-            v[j] = v[j] > 0.0 ? v[j] : 0.0;
-            if (s & 1) v[j] = 0.0;  // count each head once
-        }
-    }
-    // reduce-scatter over the 8 lanes of an octet: lane ends with position j = s >> 1
-    const bool h2 = s & 4, h1 = s & 2;
-    const double s0 = h2 ? v[0] : v[2], s1 = h2 ? v[1] : v[3];
-    const double k0 = h2 ? v[2] : v[0], k1 = h2 ? v[3] : v[1];
-    const double w0 = k0 + __shfl_xor_sync(0xffffffffu, s0, 4);
-    const double w1 = k1 + __shfl_xor_sync(0xffffffffu, s1, 4);
-    const double snd = h1 ? w0 : w1, kp = h1 ? w1 : w0;
-    double x = kp + __shfl_xor_sync(0xffffffffu, snd, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    const int j = s >> 1;
-    const int u = j >> 1;
-    const int64_t pos = (int64_t)blk[u] * kBS + (j & 1) * 4 + m;
-    const bool valid = pv[j];
-    const unsigned long long key = valid ? score_key(x) : 0ull;
-    admit(M, S, valid && (s & 1) == 0 && key >= thr, key, (int)pos);
-    if (bmax_row) {
-        // block maxima: unit u on lanes with (s >> 2) == u; reduce over m (xor 8, 16) and bit 1 (xor 2)
+    const long long keep = b0 ? w2[1] : w2[0], send = b0 ? w2[0] : w2[1];
+    const long long x = keep + shfl_xor_s64(send, 1);
+    // position of this lane
+    const int u = s >> 1, idx = (s & 1) * 4 + m;
+    const int pk = __shfl_sync(0xffffffffu, packed, u);
+    const int blk = pk >> 4, nv = pk & 15;
+    const bool valid = blk >= 0 && idx < nv;
+    const unsigned long long key = valid ? ((unsigned long long)x ^ 0x8000000000000000ull) : 0ull;
+    admit(B, S, valid && key >= thr, key, blk * kBS + idx);
+    if (bmax_row) {  // unit u on lanes s in {2u, 2u+1}, all m
         unsigned long long bm = key;
-        unsigned long long o = shfl_xor_u64(bm, 2); bm = o > bm ? o : bm;
+        unsigned long long o = shfl_xor_u64(bm, 1); bm = o > bm ? o : bm;
         o = shfl_xor_u64(bm, 8); bm = o > bm ? o : bm;
         o = shfl_xor_u64(bm, 16); bm = o > bm ? o : bm;
-        if (m == 0 && (s & 3) == 0 && uvalid[u]) bmax_row[unitA + u] = bm;
+        if (m == 0 && (s & 1) == 0 && blk >= 0) bmax_row[ustep + u] = bm;
     }
 }
 
-// ---- final merge of one row --------------------------------------------------------------------
 __device__ void stream_select_global(const unsigned long long* gk, const int* gp, int n, unsigned long long tau,
-                                     int K, Smem& M, SmemScalars& S, bool pos_is_index) {
-    if (threadIdx.x == 0) { S.nkeep = 0; S.nnew = 0; S.cur = 0; S.thr = 0; }
+                                     int K, SelBuf& B, unsigned int* hist, Scal& S, bool pos_is_index) {
+    if (threadIdx.x == 0) { S.nkeep = 0; S.nnew = 0; S.cur = 0; S.thr = tau; }
     __syncthreads();
     for (int base = 0; base < n; base += kNewCap) {
-        const unsigned long long thr = S.thr > tau ? S.thr : tau;
+        const unsigned long long thr = S.thr;
         const int cnt = min(kNewCap, n - base);
         for (int i0 = 0; i0 < cnt; i0 += kThreads) {
             const int i = i0 + threadIdx.x;
@@ -415,32 +490,38 @@ __device__ void stream_select_global(const unsigned long long* gk, const int* gp
             if (i < cnt) {
                 key = gk[base + i];
                 p = pos_is_index ? base + i : gp[base + i];
-                v = key >= thr;
+                v = key >= thr && key != 0ull;
             }
-            admit(M, S, v, key, p);
+            admit(B, S, v, key, p);
         }
         __syncthreads();
-        flush(M, S, K);
+        flush(B, hist, S, K);
     }
 }
 
 template <bool RELU>
-__global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    __shared__ __align__(16) SmemScalars S;
-    Smem M;
+__global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ Scal S;
+    __shared__ unsigned int hist[256];
+    __shared__ int kf_lut[256];
+    const int K = a.plan.k;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // shared memory: staging ring | keep[2] | new   (the merge of a pool reuses the staging ring)
+    unsigned char* staging = smem;
+    SelBuf B;
     {
-        const int kcap = max(a.plan.k, a.plan.pool_blocks);
-        unsigned char* p = smem_raw;
-        M.kcap = kcap;
-        M.keep_key[0] = reinterpret_cast<unsigned long long*>(p); p += 8 * kcap;
-        M.keep_key[1] = reinterpret_cast<unsigned long long*>(p); p += 8 * kcap;
-        M.new_key = reinterpret_cast<unsigned long long*>(p); p += 8 * kNewCap;
-        M.keep_pos[0] = reinterpret_cast<int*>(p); p += 4 * kcap;
-        M.keep_pos[1] = reinterpret_cast<int*>(p); p += 4 * kcap;
-        M.new_pos = reinterpret_cast<int*>(p); p += 4 * kNewCap;
-        M.hist = reinterpret_cast<unsigned int*>(p);
+        unsigned char* p = smem + kStagingBytes;
+        B.keep_key[0] = reinterpret_cast<unsigned long long*>(p); p += 8 * K;
+        B.keep_key[1] = reinterpret_cast<unsigned long long*>(p); p += 8 * K;
+        B.new_key = reinterpret_cast<unsigned long long*>(p); p += 8 * kNewCap;
+        B.keep_pos[0] = reinterpret_cast<int*>(p); p += 4 * K;
+        B.keep_pos[1] = reinterpret_cast<int*>(p); p += 4 * K;
+        B.new_pos = reinterpret_cast<int*>(p);
     }
+    kf_lut[tid] = e4m3_fixed(tid);
+    __syncthreads();
+
     unsigned char* ws = a.ws;
     uint32_t* status = reinterpret_cast<uint32_t*>(ws + kHdrStatus);
     unsigned int* next = reinterpret_cast<unsigned int*>(ws + kHdrIndexNext);
@@ -449,10 +530,10 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
     unsigned long long* cand_key = reinterpret_cast<unsigned long long*>(ws + a.L.cand_key);
     int* cand_pos = reinterpret_cast<int*>(ws + a.L.cand_pos);
     unsigned long long* bmax = reinterpret_cast<unsigned long long*>(ws + a.L.bmax);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int K = a.plan.k;
-    const int total = a.plan.rows * a.plan.chunks;
+    const int rows = a.plan.rows;
+    const int total = rows * a.plan.chunks;
     const bool pool = a.plan.pool_blocks > 0;
+    unsigned char* wst = staging + warp * kStages * kStepBytes;
 
     for (;;) {
         if (tid == 0) S.misc = (int)atomicAdd(next, 1u);
@@ -460,77 +541,106 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
         const int item = S.misc;
         __syncthreads();
         if (item >= total) break;
-        const int row = item / a.plan.chunks;
-        const int chunk = item % a.plan.chunks;
+        const int chunk = item / rows;
+        const int row = item % rows;
         const RowInfo R = row_info(a, row);
+        RowCtr* rc = rctr + row;
         if (!R.ok && chunk == 0 && tid == 0) set_status(status, CSA2_DEV_BAD_POS);
         const int u0 = chunk * a.plan.chunk_units;
         const int u1 = min(u0 + a.plan.chunk_units, R.n_units);
-        if (tid == 0) { S.nkeep = 0; S.nnew = 0; S.cur = 0; S.thr = 0; }
+        if (tid == 0) {
+            S.nkeep = 0; S.nnew = 0; S.cur = 0;
+            S.thr = *(volatile unsigned long long*)&rc->tau;  // lower bound left by earlier chunks
+        }
         if (u0 < u1) {
-            quantize_query(a.idx_q + (size_t)row * (kHI * kDI), S);
+            quantize_query(a.idx_q + (size_t)row * (kHI * kDI), S, kf_lut);
             __syncthreads();
-            // this lane's 32 query channels: bytes 16 s .. 16 s + 15 of the code array
+            // query words per channel chunk s and word i: 2q of channels 8i..8i+3, 8i+4..8i+7, negated
+            if (tid < 128) {
+                const int cs = tid >> 4, wi = (tid >> 2) & 3, kind = tid & 3;
+                const uint32_t cw = *reinterpret_cast<const uint32_t*>(&S.qcode[16 * cs + 4 * wi]);
+                uint32_t r = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t vq = e2m1_int2((cw >> (4 * j + ((kind & 1) ? 16 : 0))) & 15);
+                    if (kind & 2) vq = (0u - vq) & 0xFF;
+                    r |= vq << (8 * j);
+                }
+                S.qv[tid] = r;
+            }
+            __syncthreads();
             const int s = lane & 7;
-            uint32_t qh[16];
-            {
-                const uint4 c = *reinterpret_cast<const uint4*>(&S.qcode[16 * s]);
-                uint32_t t4[4];
-                e2m1x8_to_h2x4(c.x, t4); qh[0] = t4[0]; qh[1] = t4[1]; qh[2] = t4[2]; qh[3] = t4[3];
-                e2m1x8_to_h2x4(c.y, t4); qh[4] = t4[0]; qh[5] = t4[1]; qh[6] = t4[2]; qh[7] = t4[3];
-                e2m1x8_to_h2x4(c.z, t4); qh[8] = t4[0]; qh[9] = t4[1]; qh[10] = t4[2]; qh[11] = t4[3];
-                e2m1x8_to_h2x4(c.w, t4); qh[12] = t4[0]; qh[13] = t4[1]; qh[14] = t4[2]; qh[15] = t4[3];
+            uint32_t qv[16];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 q4 = *reinterpret_cast<const uint4*>(&S.qv[16 * s + 4 * i]);
+                qv[4 * i + 0] = q4.x; qv[4 * i + 1] = q4.y; qv[4 * i + 2] = q4.z; qv[4 * i + 3] = q4.w;
             }
-            const float qs0 = S.qscale[2 * s], qs1 = S.qscale[2 * s + 1];
+            const int qf0 = S.qf[2 * s], qf1 = S.qf[2 * s + 1];
             unsigned long long* bmax_row = (pool && !a.reindex) ? bmax + (size_t)row * a.plan.units_max : nullptr;
-            for (int sub = u0; sub < u1; sub += kSubUnits) {
-                const int se = min(sub + kSubUnits, u1);
-                const unsigned long long thr = S.thr;
-                for (int ua = sub + 2 * warp; ua < se; ua += 2 * kWarps)
-                    score_pair<RELU>(a, R, ua, se, qh, qs0, qs1, M, S, thr, bmax_row, status);
-                __syncthreads();
-                flush(M, S, K);
+            // every warp runs the same number of steps; step i of warp w covers units
+            // u0 + 32 i + 4 w .. +3; a selection flush follows every kStepsPerFlush steps
+            const int nsteps = (u1 - u0 + kWarps * kUnitsPerStep - 1) / (kWarps * kUnitsPerStep);
+            static_assert(kStages == 2, "two staging slots");
+            int pk0 = stage_step(a, R, u0 + kUnitsPerStep * warp, u1, wst, status), pk1 = -16;
+            cp_async_commit();
+            unsigned long long thr = S.thr;
+            for (int i = 0; i < nsteps; ++i) {
+                const int nx = i + 1;
+                if (nx < nsteps) {
+                    const int p = stage_step(a, R, u0 + kWarps * kUnitsPerStep * nx + kUnitsPerStep * warp, u1,
+                                             wst + (nx & 1) * kStepBytes, status);
+                    if (nx & 1) pk1 = p; else pk0 = p;
+                }
+                cp_async_commit();
+                cp_async_wait<kStages - 1>();
+                __syncwarp();
+                score_step<RELU>(wst + (i & 1) * kStepBytes, (i & 1) ? pk1 : pk0,
+                                 u0 + kWarps * kUnitsPerStep * i + kUnitsPerStep * warp, qv, qf0, qf1, kf_lut, B, S,
+                                 thr, bmax_row);
+                __syncwarp();
+                if ((i + 1) % kStepsPerFlush == 0 || i + 1 == nsteps) {
+                    __syncthreads();
+                    flush(B, hist, S, K);
+                    thr = S.thr;
+                }
             }
+            cp_async_wait<0>();
         }
         __syncthreads();
         // publish the local Top-k: raise the row's threshold, then emit entries >= it
-        RowCtr* rc = rctr + row;
         if (tid == 0) {
-            unsigned long long mine = (S.nkeep >= K) ? S.thr : 0ull;
-            if (mine) atomicMax(&rc->tau, mine);
+            if (S.nkeep >= K && S.thr) atomicMax(&rc->tau, S.thr);
             S.prefix = atomicAdd(&rc->tau, 0ull);
         }
         __syncthreads();
         const unsigned long long tau = S.prefix;
         const int cur = S.cur, nk = S.nkeep;
         int cnt_local = 0;
-        for (int i = tid; i < nk; i += kThreads) cnt_local += (M.keep_key[cur][i] >= tau);
-        // block-wide sum
+        for (int i = tid; i < nk; i += kThreads) cnt_local += (B.keep_key[cur][i] >= tau);
         for (int o = 16; o > 0; o >>= 1) cnt_local += __shfl_xor_sync(0xffffffffu, cnt_local, o);
-        if (lane == 0) M.hist[warp] = cnt_local;
+        if (lane == 0) hist[warp] = cnt_local;
         __syncthreads();
         if (tid == 0) {
             int tot = 0;
-            for (int w2 = 0; w2 < kWarps; ++w2) tot += M.hist[w2];
+            for (int w2 = 0; w2 < kWarps; ++w2) tot += hist[w2];
             S.misc = tot ? (int)atomicAdd(&rc->ncand, (unsigned)tot) : 0;
-            S.last = 0;
+            S.above = 0;
         }
         __syncthreads();
         {
             const size_t cbase = (size_t)row * a.plan.cand_cap + S.misc;
-            if (tid == 0) S.above = 0;
-            __syncthreads();
             for (int base = 0; base < nk; base += kThreads) {
                 const int i = base + tid;
-                const bool v = i < nk && M.keep_key[cur][i] >= tau;
+                const bool v = i < nk && B.keep_key[cur][i] >= tau;
                 const unsigned int bal = __ballot_sync(0xffffffffu, v);
                 int wb = 0;
                 if (lane == 0 && bal) wb = atomicAdd(&S.above, __popc(bal));
                 wb = __shfl_sync(0xffffffffu, wb, 0);
                 if (v) {
                     const size_t o = cbase + wb + __popc(bal & ((1u << lane) - 1));
-                    cand_key[o] = M.keep_key[cur][i];
-                    cand_pos[o] = M.keep_pos[cur][i];
+                    cand_key[o] = B.keep_key[cur][i];
+                    cand_pos[o] = B.keep_pos[cur][i];
                 }
             }
         }
@@ -544,11 +654,11 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
         const unsigned int ncand = *(volatile unsigned int*)&rc->ncand;
         const unsigned long long tau_f = *(volatile unsigned long long*)&rc->tau;
         stream_select_global(cand_key + (size_t)row * a.plan.cand_cap, cand_pos + (size_t)row * a.plan.cand_cap,
-                             (int)ncand, tau_f, K, M, S, false);
+                             (int)ncand, tau_f, K, B, hist, S, false);
         {
             const int n = S.nkeep, c = S.cur;
-            int* buf = M.new_pos;
-            for (int i = tid; i < n; i += kThreads) buf[i] = M.keep_pos[c][i];
+            int* buf = reinterpret_cast<int*>(B.keep_key[c ^ 1]);  // 2K ints >= next power of two of n
+            for (int i = tid; i < n; i += kThreads) buf[i] = B.keep_pos[c][i];
             __syncthreads();
             sort_ascending(buf, n);
             int32_t* out = a.out_idx + (size_t)row * K;
@@ -557,10 +667,18 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
         }
         if (pool && !a.reindex) {
             const int P = a.plan.pool_blocks;
-            stream_select_global(bmax + (size_t)row * a.plan.units_max, nullptr, R.n_units, 0ull, P, M, S, true);
+            SelBuf PB;  // the staging ring is idle during a merge: pool buffers live there
+            unsigned char* p = staging;
+            PB.keep_key[0] = reinterpret_cast<unsigned long long*>(p); p += 8 * P;
+            PB.keep_key[1] = reinterpret_cast<unsigned long long*>(p); p += 8 * P;
+            PB.keep_pos[0] = reinterpret_cast<int*>(p); p += 4 * P;
+            PB.keep_pos[1] = reinterpret_cast<int*>(p);
+            PB.new_key = B.new_key;
+            PB.new_pos = B.new_pos;
+            stream_select_global(bmax + (size_t)row * a.plan.units_max, nullptr, R.n_units, 0ull, P, PB, hist, S, true);
             const int n = S.nkeep, c = S.cur;
-            int* buf = M.new_pos;
-            for (int i = tid; i < n; i += kThreads) buf[i] = M.keep_pos[c][i];
+            int* buf = reinterpret_cast<int*>(PB.keep_key[c ^ 1]);
+            for (int i = tid; i < n; i += kThreads) buf[i] = PB.keep_pos[c][i];
             __syncthreads();
             sort_ascending(buf, n);
             int32_t* outp = a.out_pool + (size_t)R.b * P;
@@ -571,7 +689,6 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
         if (tid == 0) { rc->ticket = 0; rc->ncand = 0; rc->tau = 0; }
         __syncthreads();
     }
-    // last CTA out clears the work counters
     if (tid == 0) {
         __threadfence();
         if (atomicAdd(done, 1u) == gridDim.x - 1) {
@@ -583,8 +700,7 @@ __global__ void __launch_bounds__(kThreads) index_kernel(IndexArgs a) {
 }
 
 size_t smem_bytes(const IndexPlan& p) {
-    const int kcap = p.k > p.pool_blocks ? p.k : p.pool_blocks;
-    return (size_t)12 * (2 * kcap + kNewCap) + 4 * 256;
+    return (size_t)kStagingBytes + (size_t)12 * (2 * p.k + kNewCap);
 }
 
 }  // namespace

@@ -91,7 +91,7 @@ typedef struct {
     uint8_t* ik_data;
     uint8_t* ik_scale;
     uint8_t* swa;
-    int64_t cap;      /* positions per sequence in the main and indexer planes */
+    int64_t cap;      /* positions per sequence in the main and indexer planes (<= 2^30) */
     int64_t swa_cap;  /* ring slots per sequence, power of two, >= win (decode) */
 } csa2_cache;
 

@@ -39,6 +39,7 @@ def _check_rows(out, out_f32, lse, refs, tol):
 
 @pytest.mark.parametrize("B,n,k,sigma,swa_begin", [
     (3, 300, 64, 1.0, None),
+    (4, 100, 64, 1.0, None),  # 50 selected keys: a tile mixes FP4 rows and FP8 window rows
     (2, 5000, 512, 1.0, [4900, 0]),
     (300, 700, 512, 1.0, None),
     (2, 3000, 512, 8.0, None),
