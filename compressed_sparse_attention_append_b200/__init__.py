@@ -34,7 +34,7 @@ EXPORTS = (
     "csa2_entry_bytes", "csa2_status_string", "csa2_version", "csa2_workspace_size", "csa2_workspace_init",
     "csa2_quantize_append", "csa2_index_topk_full", "csa2_index_topk_reindex", "csa2_sparse_attend",
     "csa2_decode_full", "csa2_decode_reindex", "csa2_decode_minimal", "csa2_prefill_chunk",
-    "csa2_get_device_status",
+    "csa2_get_device_status", "csa2_sparse_attend_noalloc",
 )
 
 
@@ -83,6 +83,7 @@ def lib():
             "csa2_decode_minimal": (i, [S, C, i, vp, vp, vp, vp, i, vp, f, vp, vp, vp, vp, sz, vp]),
             "csa2_prefill_chunk": (i, [S, C, i64, i, vp, vp, vp, vp, vp, i, vp, i64, f, vp, vp, vp, u32, vp, sz, vp]),
             "csa2_get_device_status": (i, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
+            "csa2_sparse_attend_noalloc": (i, [S, C, i, i, vp, vp, vp, i, vp, f, vp, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -215,6 +216,14 @@ def csa2_sparse_attend(shape, cache: Cache, batch, tq, qpos, q, idx, k, out, swa
     _check("csa2_sparse_attend", lib().csa2_sparse_attend(
         ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
         _bits(out), _p(out_f32), _p(lse), ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def csa2_sparse_attend_noalloc(shape, cache: Cache, batch, tq, qpos, q, idx, k, out, swa_begin=None, sm_scale=0.0,
+                               out_f32=None, lse=None, stream=None):
+    """csa2_sparse_attend without a workspace (scratch in a static device array inside libcsa2)."""
+    _check("csa2_sparse_attend_noalloc", lib().csa2_sparse_attend_noalloc(
+        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
+        _bits(out), _p(out_f32), _p(lse), _stream(stream)))
 
 
 def csa2_decode_full(shape, cache: Cache, batch, qpos, kv, idx_k, swa_kv, idx_q, q, k, out_idx, out, pool_blocks=0,

@@ -236,6 +236,26 @@ CSA2_API csa2_status csa2_prefill_chunk(const csa2_shape* shape, const csa2_cach
                                int64_t swa_begin, float sm_scale, uint16_t* out, float* out_f32, float* lse,
                                uint32_t flags, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Sparse attention that allocates nothing and takes no workspace (the pages have no counterpart:
+ * this is a deployment convenience). Same arguments, outputs and semantics as
+ * csa2_sparse_attend, minus `ws` / `ws_bytes`. For callers that cannot allocate device memory
+ * where they run attention: a host application whose own allocator owns all device memory, or a
+ * serving loop that must not allocate after start-up because an allocation can synchronise the
+ * device.
+ *   - Scratch: a 4 MiB file-scope device array per GPU, held until the process exits.
+ *   - Limit: batch * tq <= 1024; larger calls return CSA2_ERR_CAPACITY.
+ *   - The first call on a device takes the array's device address (cudaGetSymbolAddress) and
+ *     zeroes it with a synchronous cudaMemset; make that first call before any stream capture.
+ *   - Every call shares the one array: calls whose kernels overlap on the GPU (other streams,
+ *     other threads) race and must be serialised by the caller.
+ *   - Device-side status bits (bad indices) are not reported; bad indices are still skipped.
+ */
+CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
+                                                const int64_t* qpos, const uint16_t* q, const int32_t* idx, int k,
+                                                const int64_t* swa_begin, float sm_scale, uint16_t* out,
+                                                float* out_f32, float* lse, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word in `ws`.
  * *host_status receives the CSA2_DEV_* bits; returns CSA2_ERR_DEVICE if any bit was set. */
 CSA2_API csa2_status csa2_get_device_status(void* ws, void* stream, int32_t* host_status /* host */);

@@ -25,7 +25,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_symbols()
-    assert len(names) == 14
+    assert len(names) == 15
     assert set(names) == set(csa.EXPORTS)
     for n in names:
         assert hasattr(L, n), n
