@@ -17,6 +17,7 @@ import hashlib
 import json
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -92,7 +93,9 @@ class Clocks:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # the raw samples go to $CSA2_CLOCKS_DIR when set (kept for inspection), else a temp dir
+        d = os.environ.get("CSA2_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(d, f"csa2_clocks_rank{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -167,6 +170,28 @@ def oracle_sample(wl_name, budget_s=12.0, context=None):
 # ---------------------------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------------------------
+def shard_offset(rank, batch):
+    """Weak scaling: rank r owns sequences r*batch .. r*batch+batch-1 of the global batch."""
+    return rank * batch
+
+
+def reduce_max(value, device, world):
+    """The largest of the ranks' values (every rank calls it, in the same order)."""
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_value(units_per_rank_step, world, steps, ms_max):
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return units_per_rank_step * world * steps / (ms_max / 1e3)
+
+
 def run_gpu(args):
     import torch
     import torch.distributed as dist
@@ -183,7 +208,7 @@ def run_gpu(args):
     dev = torch.device("cuda", local)
     wl = W.WORKLOADS[args.workload]
     B = args.batch or wl.batch
-    step = G.build(args.workload, batch=B, seq_offset=rank * B, context=args.context or None)
+    step = G.build(args.workload, batch=B, seq_offset=shard_offset(rank, B), context=args.context or None)
     wl = step.wl
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
@@ -226,12 +251,8 @@ def run_gpu(args):
         barrier()
     ms = start.elapsed_time(end)
     kms = {k: sum(a.elapsed_time(b) for a, b in v) / max(1, len(v)) for k, v in ev.items()}
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    queries_per_step = B * wl.tq * world
-    value = queries_per_step * args.steps / (ms_max / 1e3)
+    ms_max = reduce_max(ms, dev, world)
+    value = weak_value(B * wl.tq, world, args.steps, ms_max)
     launches = args.steps * (len(kern) if wl.mode != "minimal" else 2)
     if wl.mode == "minimal":
         kms.pop("index", None)
@@ -319,14 +340,8 @@ def run_e2e(step, args, world, barrier):
             t.copy_(step.outputs[n], non_blocking=True)
     e.record(stream)
     barrier()
-    ms = s.elapsed_time(e)
-    t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
-    v = step.batch * wl.tq * world * K / (ms / 1e3)
+    ms = reduce_max(s.elapsed_time(e), "cuda", world)
+    v = weak_value(step.batch * wl.tq, world, K, ms)
     return {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": round(ms / K, 5), "call": f"csa2_decode_{wl.mode}" if wl.mode != "prefill" else "csa2_prefill_chunk"}
 

@@ -1,6 +1,7 @@
 // abi.cu -- the extern "C" entry points of libcsa2 (declared and documented in include/csa2.h):
 // argument validation, workspace planning, kernel launches, status codes. Nothing here computes
-// any part of the layer step; every step runs in the kernels of append.cu, index.cu and attend.cu.
+// any part of the layer step; every step runs in the kernels of append.cu, index.cu, index_decode.cu
+// and attend.cu.
 #include <math.h>
 
 #include "csa2_internal.cuh"
@@ -93,7 +94,7 @@ csa2_status do_index(const csa2_shape* shape, const csa2_cache* cache, int batch
     }
     if (batch == 0) return CSA2_OK;
     const int64_t max_scan = reindex ? (int64_t)pool_stride * kBS : max_ctx;
-    IndexPlan ip = make_index_plan(batch * tq, k, max_scan, pool_blocks);
+    IndexPlan ip = make_index_plan(batch * tq, tq, k, max_scan, pool_blocks);
     WsLayout L = make_layout(&ip, nullptr);
     if (ws_bytes < L.total) return CSA2_ERR_WORKSPACE;
     IndexArgs a{};
@@ -115,7 +116,7 @@ csa2_status do_index(const csa2_shape* shape, const csa2_cache* cache, int batch
     a.plan = ip;
     a.ws = reinterpret_cast<unsigned char*>(ws);
     a.L = L;
-    return from_cuda(launch_index(a, (cudaStream_t)stream));
+    return from_cuda(ip.decode ? launch_index_decode(a, (cudaStream_t)stream) : launch_index(a, (cudaStream_t)stream));
 }
 
 csa2_status do_attend(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq, const int64_t* qpos,
@@ -187,7 +188,7 @@ csa2_status csa2_workspace_size(const csa2_shape* shape, int batch, int tq, int 
         return CSA2_ERR_INVALID_ARG;
     if ((long long)batch * tq > kMaxRows) return CSA2_ERR_INVALID_ARG;
     const int rows = batch * tq;
-    IndexPlan ip = make_index_plan(rows, k, max_scan > 0 ? max_scan : 1, pool_blocks);
+    IndexPlan ip = make_index_plan(rows, tq, k, max_scan > 0 ? max_scan : 1, pool_blocks);
     AttendPlan ap = make_attend_plan(rows, k, shape->win);
     const size_t a = index_bytes(ip), b = attend_bytes(ap);
     *bytes = a > b ? a : b;

@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
     const int g = lane >> 2, t = lane & 3;
     const int row = blockIdx.x, split = blockIdx.y;
     const int K = a.k;
+    wait_prior_grid();  // indices, cache and queries come from earlier work on the stream
     uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + kHdrStatus);
     unsigned char* qs = smem + kAWarps * kWarpSmem;
     int* list = reinterpret_cast<int*>(qs + kQBytes);
@@ -373,7 +374,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
     }
     __syncthreads();
     const int splits = a.plan.splits;
-    float* part = reinterpret_cast<float*>(a.ws + a.L.att_part) + ((size_t)row * splits) * kHQ * (kD + 2);
+    float* part = reinterpret_cast<float*>(a.ws + a.L.att_part) + ((size_t)row * splits) * kHQ * kPartStride;
     // thread -> (head h, 8 dims)
     const int h = tid >> 4, d0 = (tid & 15) * 8;
     float M = -INFINITY;
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
         for (int j = 0; j < 8; ++j) acc[j] += f * co[(w * kHQ + h) * kCoRow + 33 * (d0 >> 5) + (d0 & 31) + j];
     }
     if (splits > 1) {
-        float* pp = part + ((size_t)split * kHQ + h) * (kD + 2);
+        float* pp = part + ((size_t)split * kHQ + h) * kPartStride;
 #pragma unroll
         for (int j = 0; j < 8; ++j) pp[d0 + j] = acc[j];
         if ((tid & 15) == 0) { pp[kD] = M; pp[kD + 1] = Lsum; }
@@ -402,18 +403,31 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
         __syncthreads();
         if (!s_last) return;
         __threadfence();
-        M = -INFINITY;
-        for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, ((volatile float*)part)[((size_t)sp * kHQ + h) * (kD + 2) + kD]);
-        Lsum = 0.f;
+        // the other splits' partials, read from L2 (they were written by other CTAs); this split's
+        // own partial is still in registers
+        const float M_own = M, L_own = Lsum;
+        float acc_own[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+        for (int j = 0; j < 8; ++j) { acc_own[j] = acc[j]; acc[j] = 0.f; }
+        M = M_own;
+        for (int sp = 0; sp < splits; ++sp)
+            if (sp != split) M = fmaxf(M, __ldcg(part + ((size_t)sp * kHQ + h) * kPartStride + kD));
+        {
+            const float f = (M_own == -INFINITY) ? 0.f : exp2f(M_own - M);
+            Lsum = f * L_own;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = f * acc_own[j];
+        }
         for (int sp = 0; sp < splits; ++sp) {
-            const volatile float* q = part + ((size_t)sp * kHQ + h) * (kD + 2);
-            const float mw = q[kD];
+            if (sp == split) continue;
+            const float* q = part + ((size_t)sp * kHQ + h) * kPartStride;
+            const float4 v0 = __ldcg(reinterpret_cast<const float4*>(q + d0));
+            const float4 v1 = __ldcg(reinterpret_cast<const float4*>(q + d0 + 4));
+            const float mw = __ldcg(q + kD), lw = __ldcg(q + kD + 1);
             const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-            Lsum += f * q[kD + 1];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] += f * q[d0 + j];
+            Lsum += f * lw;
+            acc[0] += f * v0.x; acc[1] += f * v0.y; acc[2] += f * v0.z; acc[3] += f * v0.w;
+            acc[4] += f * v1.x; acc[5] += f * v1.y; acc[6] += f * v1.z; acc[7] += f * v1.w;
         }
         if (tid == 0) *tk = 0;
     }
@@ -443,8 +457,7 @@ cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     if (a.rows == 0) return cudaSuccess;
     dim3 grid(a.rows, a.plan.splits);
-    attend_kernel<<<grid, kAThreads, smem, s>>>(a);
-    return cudaGetLastError();
+    return launch_after_prior(attend_kernel, grid, dim3(kAThreads), smem, s, a);
 }
 
 }  // namespace csa2

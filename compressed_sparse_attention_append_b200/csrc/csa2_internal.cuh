@@ -30,6 +30,7 @@ constexpr int kIKScales = kHK * kDI / 16; // 16
 constexpr int kBS = 8;        // positions per pool block
 constexpr int kSWABytes = 256;
 constexpr int kMaxK = 2048;   // largest Top-k / pool size
+constexpr int kPartStride = kD + 4;  // floats per (split, head) partial: O[128], m, l, 2 pad (16-byte rows)
 
 // ---- device status word (first 4 bytes of the workspace) --------------------------------------
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
@@ -91,6 +92,28 @@ __device__ __forceinline__ uint64_t score_key(double s) {
     return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
+// ---- programmatic dependent launch -----------------------------------------------------------------
+// Kernels that read an earlier kernel's output are launched with programmatic stream serialisation,
+// so that their launch overlaps the end of the kernel before them; each one waits here before its
+// first access to data an earlier kernel wrote (a no-op when launched without the attribute).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_after_prior(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                      Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- cp.async helpers ----------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
     uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
@@ -115,6 +138,7 @@ struct IndexPlan {
     int chunks;        // work items per row
     int pool_blocks;   // 0 = no pool
     size_t cand_cap;   // candidate slots per row
+    int decode;        // 1: one query row per sequence, scored by score_kernel then select_kernel
 };
 
 struct AttendPlan {
@@ -131,6 +155,11 @@ struct AttendPlan {
 //   [.., +4*kMaxRows)   attention ticket per row
 //   data: candidates, block maxima, attention partials (contents are scratch)
 constexpr int kMaxRows = 65536;
+constexpr int kKeyBins = 2048;  // score histogram bins of a decode row (sign, exponent, 4 mantissa bits)
+constexpr int kSelCand = 4096;  // candidates of a decode row ranked by its last select CTA
+constexpr int kSubBins = 1024;  // second-level bins (the next 10 bits) of a decode row's cut bin
+// per decode row: key histogram, block-maximum histogram, and the two second-level histograms
+constexpr int kRowHist = 2 * (kKeyBins + kSubBins);
 constexpr size_t kHdrStatus = 0, kHdrIndexNext = 8, kHdrIndexDone = 12;
 
 struct WsLayout {
@@ -139,19 +168,40 @@ struct WsLayout {
     size_t cand_key;   // u64[rows * cand_cap]
     size_t cand_pos;   // i32[rows * cand_cap]
     size_t bmax;       // u64[rows * units_max] (pool)
-    size_t att_part;   // f32[rows * splits * hq * (d + 2)]
+    size_t key_hist;   // u32[rows][kRowHist] (decode plans: score histograms)
+    size_t sel_key;    // u64[rows][2][kSelCand] (decode plans: candidate keys, then block maxima)
+    size_t sel_pos;    // u64[rows][2][kSelCand] (element index << 32 | position, of each candidate)
+    size_t att_part;   // f32[rows * splits * hq * kPartStride]
     size_t total;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline IndexPlan make_index_plan(int rows, int k, int64_t max_scan, int pool_blocks) {
+// RowCtr index stride of the decode index path: row r uses RowCtr[r * stride], a 128-byte line of
+// its own when the rows allow it (atomics of different rows then never share a line).
+__host__ __device__ inline int ctr_stride(int rows) { return rows <= kMaxRows / 8 ? 8 : 1; }
+
+inline IndexPlan make_index_plan(int rows, int tq, int k, int64_t max_scan, int pool_blocks) {
     IndexPlan p{};
     p.rows = rows;
     p.k = k;
     p.pool_blocks = pool_blocks;
     p.units_max = (int)((max_scan + kBS - 1) / kBS);
     if (p.units_max < 1) p.units_max = 1;
+    if (tq == 1) {
+        // decode rows: every position's key is stored (8 bytes against 144 bytes of indexer entry),
+        // work items of chunk_units units sized for about 4 items per resident warp (148 SMs x 16)
+        p.decode = 1;
+        const long long units = (long long)rows * p.units_max;
+        long long cu = (units + 148 * 16 * 4 - 1) / (148 * 16 * 4);
+        cu = (cu + 3) / 4 * 4;
+        if (cu < 16) cu = 16;
+        if (cu > 512) cu = 512;
+        p.chunk_units = (int)cu;
+        p.chunks = (p.units_max + p.chunk_units - 1) / p.chunk_units;
+        p.cand_cap = (size_t)p.units_max * kBS;
+        return p;
+    }
     const int items_target = 148 * 4;
     int chunks_target = (items_target + rows - 1) / rows;
     if (chunks_target < 1) chunks_target = 1;
@@ -189,16 +239,21 @@ inline WsLayout make_layout(const IndexPlan* ip, const AttendPlan* ap) {
     int rows_i = ip ? ip->rows : 0;
     size_t cc = ip ? ip->cand_cap : 0;
     L.cand_key = off; off = align256(off + 8 * (size_t)rows_i * cc);
-    L.cand_pos = off; off = align256(off + 4 * (size_t)rows_i * cc);
-    size_t bm = (ip && ip->pool_blocks > 0) ? (size_t)rows_i * (size_t)ip->units_max : 0;
+    L.cand_pos = off; off = align256(off + ((ip && ip->decode) ? 0 : 4 * (size_t)rows_i * cc));
+    // rows of the decode path start on 16-byte boundaries (an even number of u64 per row)
+    size_t bm = (ip && ip->pool_blocks > 0) ? (size_t)rows_i * (size_t)((ip->units_max + 1) & ~1) : 0;
     L.bmax = off; off = align256(off + 8 * bm);
-    size_t part = ap ? (size_t)ap->rows * (size_t)ap->splits * kHQ * (kD + 2) : 0;
+    const size_t drows = (ip && ip->decode) ? (size_t)rows_i : 0;
+    L.key_hist = off; off = align256(off + drows * kRowHist * 4);
+    L.sel_key = off; off = align256(off + drows * 2 * kSelCand * 8);
+    L.sel_pos = off; off = align256(off + drows * 2 * kSelCand * 8);
+    size_t part = ap ? (size_t)ap->rows * (size_t)ap->splits * kHQ * kPartStride : 0;
     L.att_part = off; off = align256(off + 4 * part);
     L.total = off;
     return L;
 }
 
-// ---- kernel launchers (defined in append.cu, index.cu, attend.cu) -----------------------------------
+// ---- kernel launchers (defined in append.cu, index.cu, index_decode.cu, attend.cu) -----------------------------------
 struct AppendArgs {
     csa2_cache c;
     int batch, t;
@@ -231,7 +286,8 @@ struct IndexArgs {
     unsigned char* ws;
     WsLayout L;
 };
-cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);
+cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);         // index.cu: any tq
+cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s);  // index_decode.cu: plan.decode
 
 struct AttendArgs {
     csa2_cache c;

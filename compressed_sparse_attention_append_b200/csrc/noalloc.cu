@@ -73,7 +73,7 @@ extern "C" CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* sha
     WsLayout L{};
     L.att_ticket = kNoAllocTickets;
     L.att_part = kNoAllocParts;
-    const size_t part = ap.splits > 1 ? (size_t)ap.rows * ap.splits * kHQ * (kD + 2) * 4 : 0;
+    const size_t part = ap.splits > 1 ? (size_t)ap.rows * ap.splits * kHQ * kPartStride * 4 : 0;
     if (kNoAllocParts + part > kNoAllocBytes) return CSA2_ERR_CAPACITY;
     void* scratch = nullptr;
     csa2_status st = noalloc_scratch(&scratch);

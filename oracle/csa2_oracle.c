@@ -18,9 +18,26 @@
  * decisions equal those of exact rational arithmetic. Index scores are sums of products
  * that are multiples of 2^-20 with magnitude below 2^31, so fp64 sums are exact in any order.
  *
- * Readings of the pages that the sources leave open (scale rule, rounding, score formula,
- * tie-break, layout, softmax structure) are listed in the design doc as R1..R12 and marked
- * "(Rn)" where they are applied.
+ * Readings of the pages where the sources leave a step open; "(Rn)" marks where each applies:
+ *   R1  scale s = E4M3_RNE_satfinite(amax / 6); s == 0 gives all-zero codes; element code =
+ *       E2M1_RNE_satfinite(x / s), sign kept (a negative value rounding to 0 gives code 0x8).
+ *   R2  index score = sum over the 4 indexer heads of q_h . k_h on dequantised values; with the
+ *       ReLU flag, sum over heads of max(0, q_h . k_h).
+ *   R3  4 indexer key heads of 64 channels; query head h uses key head h * hk / hi.
+ *   R4  the indexer query is quantised with the R1 codec before scoring.
+ *   R5  ranking by score descending, ties to the lower position (lower block id for the pool).
+ *   R6  selected positions are emitted ascending; fewer than k visible -> all, padded with -1.
+ *   R7  one softmax over the selected FP4 rows and the FP8 window rows, no de-duplication,
+ *       scale 1/sqrt(128), no sink.
+ *   R8  window entries are E4M3 without a scale (RNE, satfinite); K = channels 0..127, V =
+ *       128..255; a query at i sees window positions max(s, i - 127) .. i.
+ *   R9  cache planes per sequence: packed codes (channel 2j in the low nibble of byte j) and
+ *       one scale byte per 16 channels; an entry is ch/2 + ch/16 bytes.
+ *   R10 pool = the top min(2048, ceil(N / 8)) blocks by their maximum visible score; block b
+ *       covers positions 8b .. 8b+7.
+ *   R11 a decode query sits at N - 1 and is appended before scoring (so it is visible);
+ *       prefill row i sees positions <= i.
+ *   R12 compression ratio 1: one cache entry per token.
  *
  * Parity pins: every function here is checked by tests/test_oracle_*.py against exact
  * rational arithmetic, library routines (torch float8 conversion, Python sorted(), torch

@@ -62,5 +62,7 @@ def bf16_np(t: torch.Tensor) -> np.ndarray:
 
 
 def attn_tol(oracle_out: np.ndarray, sigma: float = 1.0):
-    """Tolerance of fp32 attention against the fp64 oracle (derivation in the design doc)."""
+    """Tolerance of fp32 attention against the fp64 oracle: fp16 products of exact dequantised
+    values, fp32 accumulation of <= 2176 terms and exp2 of fp32 logits give an error well below
+    2e-3 of the output scale at unit-variance inputs; the scale grows with sigma."""
     return 2e-3 * max(1.0, sigma)

@@ -1,7 +1,7 @@
 """Sparse attention and the four per-mode compositions on the GPU against the oracle.
 
-Attention outputs (fp32) must be within the tolerance derived in the design doc (2e-3 at unit-variance
-inputs, scaled with sigma); the bf16 output must be the round-to-nearest-even of the fp32 output;
+Attention outputs (fp32) must be within 2e-3 at unit-variance inputs, scaled with sigma (the bound
+of fp16 products of exact dequantised values with fp32 accumulation); the bf16 output must be the round-to-nearest-even of the fp32 output;
 index outputs of the compositions must be identical to the oracle's.
 """
 import numpy as np

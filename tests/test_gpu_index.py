@@ -56,6 +56,100 @@ def test_full_mode_matches_oracle(orc, B, n, k, pool, sigma, ragged):
             assert np.array_equal(out[b].cpu().numpy(), ridx), (rep, b)
 
 
+def test_full_mode_multi_row_queries(orc):
+    """tq > 1 query rows per sequence (the prefill form): every row ranks its own visible prefix."""
+    B, n, tq, k = 2, 5000, 3, 256
+    seed = 91
+    shape, cache, swa_cap = _setup(B, n, seed)
+    qpos = [[n - 1 - 700 * b - 13 * t for t in range(tq)] for b in range(B)]
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV).reshape(-1)
+    rows_b = torch.arange(B).repeat_interleave(tq)
+    iq = query_values(seed, "iq", rows_b.to(DEV), qp, 256, DEV).contiguous()
+    out = torch.full((B * tq, k), -7, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, tq, k, n)
+    csa.csa2_index_topk_full(shape, cache, B, tq, qp, iq, k, out, max_ctx=n, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    for b in range(B):
+        oc = oracle_seq(seed, b, n, n, swa_cap)
+        for t in range(tq):
+            qb = query_values(seed, "iq", [b], [qpos[b][t]], 256, "cpu")[0]
+            ref = oc.index_topk_full(qpos[b][t], qb, k=k)
+            assert np.array_equal(out[b * tq + t].cpu().numpy(), ref), (b, t)
+
+
+def test_full_mode_long_pool(orc):
+    """More pool blocks than fit on chip (17,500 blocks of 8): the pool ranking reads from memory."""
+    B, n, k, P = 1, 140000, 64, 256
+    seed = 17
+    shape, cache, swa_cap = _setup(B, n, seed, cap=n)
+    qp = torch.tensor([n - 1], dtype=torch.int64, device=DEV)
+    iq = query_values(seed, "iq", [0], qp, 256, DEV).contiguous()
+    out = torch.empty(B, k, dtype=torch.int32, device=DEV)
+    opool = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    opn = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, n, P)
+    csa.csa2_index_topk_full(shape, cache, B, 1, qp, iq, k, out, P, opool, opn, max_ctx=n, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    oc = oracle_seq(seed, 0, n, n, swa_cap)
+    qb = query_values(seed, "iq", [0], [n - 1], 256, "cpu")[0]
+    ridx, rpool, rpn = oc.index_topk_full(n - 1, qb, k=k, pool_blocks=P)
+    assert int(opn[0]) == rpn
+    assert np.array_equal(opool[0].cpu().numpy(), rpool)
+    assert np.array_equal(out[0].cpu().numpy(), ridx)
+
+
+def _full_from_rows(ik_cpu, kv_cpu, k, pool=0):
+    """Full mode over one sequence whose indexer keys are the given bf16 rows (made on the host)."""
+    n = ik_cpu.shape[0]
+    shape = csa.make_shape()
+    cache = csa.Cache(1, n, 1 << max(7, (n - 1).bit_length()))
+    csa.csa2_quantize_append(shape, cache, 1, n, torch.zeros(1, dtype=torch.int64, device=DEV),
+                             kv_cpu[None].to(DEV).contiguous(), ik_cpu[None].to(DEV).contiguous(),
+                             kv_cpu[None].to(DEV).contiguous())
+    iq = query_values(5, "iq", [0], [n - 1], 256, "cpu")
+    qp = torch.tensor([n - 1], dtype=torch.int64, device=DEV)
+    out = torch.empty(1, k, dtype=torch.int32, device=DEV)
+    opool = torch.empty(1, max(pool, 1), dtype=torch.int32, device=DEV)
+    opn = torch.empty(1, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, 1, 1, k, n, pool)
+    csa.csa2_index_topk_full(shape, cache, 1, 1, qp, iq.to(DEV).contiguous(), k, out, pool,
+                             opool if pool else None, opn if pool else None, max_ctx=n, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    oc = oracle.SeqCache(n, 1 << max(7, (n - 1).bit_length()))
+    oc.append(0, kv=bf16_np(kv_cpu), idx_k=bf16_np(ik_cpu))
+    if pool:
+        ridx, rpool, rpn = oc.index_topk_full(n - 1, bf16_np(iq[0]), k=k, pool_blocks=pool)
+        assert int(opn[0]) == rpn
+        assert np.array_equal(opool[0].cpu().numpy(), rpool)
+    else:
+        ridx = oc.index_topk_full(n - 1, bf16_np(iq[0]), k=k)
+    got = out[0].cpu().numpy()
+    assert np.array_equal(got, ridx)
+    return got
+
+
+def test_full_mode_all_keys_equal(orc):
+    """Every position has the same indexer key: one score for all, so the k lowest positions win."""
+    n, k = 5000, 256
+    p = torch.arange(n)
+    ik = values(6, "ik", [0], torch.zeros(n, dtype=torch.int64), 256, "cpu")[0]
+    kv = values(6, "kv", [0], p, 256, "cpu")[0]
+    got = _full_from_rows(ik, kv, k, pool=64)
+    assert np.array_equal(got, np.arange(k))
+
+
+def test_full_mode_sample_blind_to_most_keys(orc):
+    """Keys at every 5th position are 8x larger: a regular sample of the keys sees only those, so the
+    threshold it suggests admits fewer than k keys and the ranking must run over every key."""
+    n, k = 20000, 512
+    p = torch.arange(n)
+    ik = values(8, "ik", [0], p, 256, "cpu")[0].float()
+    ik[p % 5 == 0] *= 8.0
+    ik = ik.to(torch.bfloat16)
+    kv = values(8, "kv", [0], p, 256, "cpu")[0]
+    _full_from_rows(ik, kv, k, pool=300)
+
+
 def test_full_mode_relu_and_ties(orc):
     """Identical indexer keys at many positions force exact score ties: the lower position wins."""
     B, n, k = 1, 3000, 512
@@ -78,12 +172,22 @@ def test_full_mode_relu_and_ties(orc):
         assert np.array_equal(out[0].cpu().numpy(), ref), relu
 
 
-@pytest.mark.parametrize("B,n,P,k", [(2, 4096, 40, 128), (3, 50000, 2000, 512), (1, 1000, 125, 512)])
-def test_reindex_matches_oracle(orc, B, n, P, k):
+@pytest.mark.parametrize("B,n,P,k,shuffled", [
+    (2, 4096, 40, 128, False),
+    (3, 50000, 2000, 512, False),
+    (1, 1000, 125, 512, False),
+    (3, 1000, 125, 64, False),   # 125 units per row: the last scoring step reaches past each row
+    (2, 5000, 301, 64, True),    # pool blocks listed out of order: the output is still ascending
+])
+def test_reindex_matches_oracle(orc, B, n, P, k, shuffled):
     seed = 23 + P
     shape, cache, swa_cap = _setup(B, n, seed)
     nblk = (n + 7) // 8
-    pool = W.distinct_sorted(seed, "pool", torch.arange(B, device=DEV), nblk, P).to(torch.int32).contiguous()
+    pool = W.distinct_sorted(seed, "pool", torch.arange(B, device=DEV), nblk, P).to(torch.int32)
+    if shuffled:
+        g = torch.Generator().manual_seed(seed)
+        pool = torch.stack([r[torch.randperm(P, generator=g).to(DEV)] for r in pool])
+    pool = pool.contiguous()
     pool_n = torch.tensor([P - 3 * i for i in range(B)], dtype=torch.int32, device=DEV)
     qpos = [n - 1 - 101 * i for i in range(B)]
     qp = torch.tensor(qpos, dtype=torch.int64, device=DEV)
