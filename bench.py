@@ -271,13 +271,15 @@ def run_gpu(args):
     dom = "index" if wl.mode in ("full", "reindex") else ("attend" if wl.mode == "minimal" else "prefill")
     if dom == "prefill":
         dom_bytes = (ab["index"] + ab["attend"]) * wl.tq
-        dom_file = "index.cu"
+        dom_file, dom_kernels = "index.cu", "index_kernel + attend_kernel"
     else:
         dom_bytes = ab[dom] * B
-        dom_file = "index.cu" if dom == "index" else "attend.cu"
+        # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
+        dom_file = "index_decode.cu" if dom == "index" else "attend.cu"
+        dom_kernels = "zero_kernel + score_kernel + select_kernel" if dom == "index" else "attend_kernel"
     dur_s = kms[dom] / 1e3
     achieved = dom_bytes / dur_s / 1e9
-    roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+    roof = {"kernel": dom, "kernels": dom_kernels, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "peak_kind": f"of {peak_kind}",
             "traffic": ncu_traffic(dom_file, args.workload), "algorithmic_bytes_per_launch": dom_bytes,
             "ms_per_launch": round(kms[dom], 5)}

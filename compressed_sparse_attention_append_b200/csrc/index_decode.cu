@@ -623,11 +623,14 @@ __device__ int cut_bin(const unsigned int* h, int nbins, int K, SelScal& S, int*
     const int per = nbins / kQThreads;  // 8 or 16
     unsigned int hb[kKeyBins / kQThreads];
     int sum = 0;
+    const uint4* hv = reinterpret_cast<const uint4*>(h + nbins - per * (tid + 1));  // 16-byte aligned
 #pragma unroll
-    for (int j = 0; j < kKeyBins / kQThreads; ++j) {
-        hb[j] = j < per ? __ldcg(h + nbins - per * (tid + 1) + j) : 0u;
-        sum += (int)hb[j];
+    for (int q = 0; q < kKeyBins / kQThreads / 4; ++q) {
+        const uint4 v = 4 * q < per ? __ldcg(hv + q) : make_uint4(0u, 0u, 0u, 0u);
+        hb[4 * q] = v.x; hb[4 * q + 1] = v.y; hb[4 * q + 2] = v.z; hb[4 * q + 3] = v.w;
     }
+#pragma unroll
+    for (int j = 0; j < kKeyBins / kQThreads; ++j) sum += (int)hb[j];
     if (tid == 0) { S.digit = -1; S.above = 0; }
     int total;
     const int excl = block_excl_scan(sum, S.wsum, total);  // its barriers order the reset above
@@ -883,17 +886,33 @@ __global__ void __launch_bounds__(kQThreads, 8) select_kernel(IndexArgs a, int s
     const int b0 = (int)((long long)nbatch * slice / slices), b1 = (int)((long long)nbatch * (slice + 1) / slices);
     // the first batch's keys are requested before anything else
     const int32_t* prow = a.reindex ? a.pool + (size_t)row * a.pool_stride : nullptr;
+    // thread t of batch bt owns unit u = bt * kQThreads + t: its 8 keys (64 contiguous bytes), its
+    // block maximum and its pool id
     unsigned long long kk[kPerT];
-    int pid[kPerT];  // pool id of each key's unit (Reindex)
-    auto load_keys = [&](int bt) {
+    int pid = 0, pid_next = 0;
+    unsigned long long bmv = 0;
+    auto load_unit = [&](int bt) {
+        const int u = bt * kQThreads + tid;
+        if (u < a.plan.units_max) {
+            const uint4* src = reinterpret_cast<const uint4*>(gk + (size_t)u * kBS);
 #pragma unroll
-        for (int j = 0; j < kPerT; ++j) {
-            const int i = bt * kBatch + j * kQThreads + tid;
-            kk[j] = i < nmax ? __ldcg(gk + i) : 0ull;
-            pid[j] = (prow && i < nmax) ? __ldg(prow + (i >> 3)) : 0;
+            for (int q = 0; q < kPerT / 2; ++q) {
+                const uint4 v = __ldcg(src + q);
+                kk[2 * q] = ((unsigned long long)v.y << 32) | v.x;
+                kk[2 * q + 1] = ((unsigned long long)v.w << 32) | v.z;
+            }
+            pid = prow ? __ldg(prow + u) : u;
+            pid_next = (prow && u + 1 < a.plan.units_max) ? __ldg(prow + u + 1) : 0x7FFFFFFF;
+            bmv = pool_on ? __ldcg(gb + u) : 0ull;
+        } else {
+#pragma unroll
+            for (int j = 0; j < kPerT; ++j) kk[j] = 0ull;
+            pid = 0;
+            pid_next = 0x7FFFFFFF;
+            bmv = 0ull;
         }
     };
-    if (b0 < b1) load_keys(b0);
+    if (b0 < b1) load_unit(b0);
     bool ok;
     const DRow R = drow(a, row, ok);
     const int n = R.n_units * kBS;
@@ -903,18 +922,17 @@ __global__ void __launch_bounds__(kQThreads, 8) select_kernel(IndexArgs a, int s
     if (pool_on) pstar = cut_bin(hrow + kKeyBins, kKeyBins, P, S, &pabove);
     int unsorted = 0;
     for (int bt = b0; bt < b1; ++bt) {
-        if (bt > b0) load_keys(bt);
-        const int u = bt * (kBatch / kBS) + tid;  // this thread's unit of the batch
-        const unsigned long long bmv = (pool_on && u < a.plan.units_max) ? __ldcg(gb + u) : 0ull;
-        if (prow && u + 1 < R.n_units) unsorted |= __ldg(prow + u) >= __ldg(prow + u + 1);
+        if (bt > b0) load_unit(bt);
+        const int u = bt * kQThreads + tid;
+        if (prow && u + 1 < R.n_units) unsorted |= pid >= pid_next;
         bool take[kPerT];
         unsigned long long ip[kPerT];
 #pragma unroll
         for (int j = 0; j < kPerT; ++j) {
-            const int i = bt * kBatch + j * kQThreads + tid;
+            const int i = u * kBS + j;
             const int b = kk[j] ? key_bin(kk[j]) : -2;
             take[j] = i < n && b >= bstar && b >= -1;
-            const int p = prow ? pid[j] * kBS + (i & 7) : i;
+            const int p = pid * kBS + j;  // Full mode: pid == u
             ip[j] = ((unsigned long long)(unsigned int)i << 32) | (unsigned int)p;
             if (take[j] && b == bstar) atomicAdd(hsub + sub_bin(kk[j]), 1u);
         }
