@@ -253,7 +253,9 @@ def run_gpu(args):
     kms = {k: sum(a.elapsed_time(b) for a, b in v) / max(1, len(v)) for k, v in ev.items()}
     ms_max = reduce_max(ms, dev, world)
     value = weak_value(B * wl.tq, world, args.steps, ms_max)
-    launches = args.steps * (len(kern) if wl.mode != "minimal" else 2)
+    # kernels per step: append 1; index (decode rows) zero + score + select = 3, (prefill) 1; attend 1
+    per_step = {"full": 5, "reindex": 5, "minimal": 2}.get(wl.mode, 3)
+    launches = args.steps * per_step
     if wl.mode == "minimal":
         kms.pop("index", None)
 
