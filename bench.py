@@ -280,11 +280,24 @@ def run_gpu(args):
         dom_file = "index_decode.cu" if dom == "index" else "attend.cu"
         dom_kernels = "zero_kernel + score_kernel + select_kernel" if dom == "index" else "attend_kernel"
     dur_s = kms[dom] / 1e3
-    achieved = dom_bytes / dur_s / 1e9
-    roof = {"kernel": dom, "kernels": dom_kernels, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "peak_kind": f"of {peak_kind}",
-            "traffic": ncu_traffic(dom_file, args.workload), "algorithmic_bytes_per_launch": dom_bytes,
-            "ms_per_launch": round(kms[dom], 5)}
+    if dom == "prefill":
+        # the prefill chunk scores every visible (row, position) pair with dp4a on the CUDA cores:
+        # bound by integer issue. Useful multiply-adds per chunk: rows x visible positions x 256
+        # channels; peak = 148 SMs x 64 dp4a lanes per clock x 4 multiply-adds x 1.965 GHz.
+        visible = wl.context - wl.tq + (wl.tq + 1) / 2.0
+        macs = wl.tq * visible * 256
+        achieved = macs / dur_s / 1e12
+        alu_peak = 148 * 64 * 4 * 1.965e9 / 1e12
+        roof = {"kernel": dom, "kernels": dom_kernels, "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(alu_peak, 1), "unit": "TMAC/s", "frac": round(achieved / alu_peak, 4),
+                "peak_kind": "derived (dp4a issue rate x clock)", "traffic": None,
+                "macs_per_launch": macs, "ms_per_launch": round(kms[dom], 5)}
+    else:
+        achieved = dom_bytes / dur_s / 1e9
+        roof = {"kernel": dom, "kernels": dom_kernels, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_kind": f"of {peak_kind}",
+                "traffic": ncu_traffic(dom_file, args.workload), "algorithmic_bytes_per_launch": dom_bytes,
+                "ms_per_launch": round(kms[dom], 5)}
     step_bytes = sum(ab.values()) * B * wl.tq
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,

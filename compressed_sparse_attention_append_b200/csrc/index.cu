@@ -1,11 +1,10 @@
-// index.cu -- indexer scoring, exact Top-k selection and the block candidate pool.
+// index.cu -- indexer scoring and exact Top-k selection for several query rows per sequence (the
+// prefill chunk: row i of a chunk sees positions <= i). Rows of one query per sequence (decode:
+// Full with its block pool, and Reindex) run in index_decode.cu.
 //
 // [B] "DeepSeek Cuts KV Cache Footprint Fourfold", "Technical Approach": Full mode computes the
-// Top-K indices; Reindex recomputes the selection inside the shared candidate pool built by the
-// decoder's first Full layer. [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890
-// Bytes per Token", sec. VI "Shortlist-of-a-shortlist" and sec. IX Figure 4: each block of 8
-// positions is scored by the maximum index score among its positions and the winning blocks (up
-// to 2,048) form the pool. sec. XI: indexer queries and keys are FP4.
+// Top-K indices. [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token",
+// sec. IX (the indexer scores every visible position), sec. XI: indexer queries and keys are FP4.
 //
 // Score (this build's reading; the pages give no formula): score(p) = sum_h q_h . k_{p,h} over 4
 // heads x 64 channels of dequantised FP4 values, computed EXACTLY as the integer S = score * 2^20:
@@ -18,18 +17,17 @@
 //     (<= 245760); D * f(s_k) fits in int32 and (D * f(s_k)) * f(s_q) is added to an int64
 //     with one wide multiply-add (each term < 2^47, the sum of 16 terms < 2^51).
 // No floating-point conversion runs in the scoring loop. Ranking is by S descending, ties to the
-// lower position (to the lower block id for the pool); S is the same integer the exact rational
-// score gives, so the selected set is unique and reproducible.
+// lower position; S is the same integer the exact rational score gives, so the selected set is
+// unique and reproducible.
 //
 // Structure (one kernel, persistent CTAs taking work items from an atomic counter):
 //   item = (chunk of 8-position units, query row), chunk-major so that later chunks of a row start
-//   with the admission threshold left by its earlier chunks. Each warp scores two units per step
-//   (16 positions, 2 KB of keys + 256 B of scales) from a private 3-stage cp.async ring; a running
+//   with the admission threshold left by its earlier chunks. Each warp scores four units per step
+//   (32 positions, 4 KB of keys + 512 B of scales) from a private 2-stage cp.async ring; a running
 //   local Top-k sits in shared memory (admission threshold + radix select over orderable keys,
 //   skipping the bits all keys share and histogramming with match_any). A CTA emits its local
 //   Top-k to the row's candidate list; the CTA that finishes a row's last chunk merges the
-//   candidates (and, for the pool, the per-unit block maxima) into the final ascending outputs
-//   and clears the row's counters.
+//   candidates into the final ascending outputs and clears the row's counters.
 #include "csa2_internal.cuh"
 
 namespace csa2 {
@@ -352,36 +350,22 @@ __device__ RowInfo row_info(const IndexArgs& a, int row) {
     r.b = row / a.tq;
     r.qpos = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
     r.ok = true;
-    if (r.qpos < 0 || r.qpos >= a.c.cap || (!a.reindex && r.qpos >= a.max_ctx)) {
+    if (r.qpos < 0 || r.qpos >= a.c.cap || r.qpos >= a.max_ctx) {
         r.ok = false;
         r.n_units = 0;
         return r;
     }
-    if (a.reindex) {
-        int n = a.pool_n[r.b];
-        if (n < 0 || n > a.pool_stride) n = n < 0 ? 0 : a.pool_stride;
-        r.n_units = n;
-    } else {
-        r.n_units = (int)((r.qpos + kBS) / kBS);
-    }
+    r.n_units = (int)((r.qpos + kBS) / kBS);
     return r;
 }
 
-// Block id of unit u of row R and its number of scoreable positions (0..8); -1 / 0 when the unit is
-// past the chunk or its pool id is invalid.
-__device__ __forceinline__ void unit_info(const IndexArgs& a, const RowInfo& R, int u, int u_end, int& blk, int& nv,
-                                          uint32_t* status) {
+// Block id of unit u of row R (the unit itself) and its number of scoreable positions (0..8);
+// -1 / 0 when the unit is past the chunk.
+__device__ __forceinline__ void unit_info(const IndexArgs& a, const RowInfo& R, int u, int u_end, int& blk, int& nv) {
     blk = -1;
     nv = 0;
     if (u >= u_end) return;
-    int id = u;
-    if (a.reindex) {
-        id = __ldg(a.pool + (size_t)R.b * a.pool_stride + u);
-        if (id < 0 || (int64_t)id * kBS >= a.c.cap) {
-            set_status(status, CSA2_DEV_BAD_POOL);
-            return;
-        }
-    }
+    const int id = u;
     const int64_t p0 = (int64_t)id * kBS;
     int64_t n = R.qpos - p0 + 1;
     if (a.c.cap - p0 < n) n = a.c.cap - p0;
@@ -393,10 +377,10 @@ __device__ __forceinline__ void unit_info(const IndexArgs& a, const RowInfo& R, 
 // One warp step: units u .. u+3. Lane u (< 4) resolves unit u; the result is broadcast.
 // Staging: codes of unit j at 1024*j, scales at 4096 + 128*j.
 __device__ __forceinline__ int stage_step(const IndexArgs& a, const RowInfo& R, int ustep, int u_end,
-                                          unsigned char* st, uint32_t* status) {
+                                          unsigned char* st) {
     const int lane = threadIdx.x & 31;
     int blk = -1, nv = 0;
-    if (lane < kUnitsPerStep) unit_info(a, R, ustep + lane, u_end, blk, nv, status);
+    if (lane < kUnitsPerStep) unit_info(a, R, ustep + lane, u_end, blk, nv);
     const int packed = (blk << 4) | nv;  // blk < 2^26 (cap <= 2^30 positions); -1 packs to -16
     const uint8_t* base = a.c.ik_data + (size_t)R.b * a.c.cap * kIKBytes;
     const uint8_t* sbase = a.c.ik_scale + (size_t)R.b * a.c.cap * kIKScales;
@@ -422,7 +406,7 @@ __device__ __forceinline__ int stage_step(const IndexArgs& a, const RowInfo& R, 
 template <bool RELU>
 __device__ __forceinline__ void score_step(const unsigned char* st, int packed, int ustep, const uint32_t (&qv)[16],
                                            int qf0, int qf1, const int* kf_lut, SelBuf& B, Scal& S,
-                                           unsigned long long thr, unsigned long long* bmax_row) {
+                                           unsigned long long thr) {
     const int lane = threadIdx.x & 31;
     const int m = lane >> 3, s = lane & 7;
     long long v[8];
@@ -466,13 +450,6 @@ __device__ __forceinline__ void score_step(const unsigned char* st, int packed, 
     const bool valid = blk >= 0 && idx < nv;
     const unsigned long long key = valid ? ((unsigned long long)x ^ 0x8000000000000000ull) : 0ull;
     admit(B, S, valid && key >= thr, key, blk * kBS + idx);
-    if (bmax_row) {  // unit u on lanes s in {2u, 2u+1}, all m
-        unsigned long long bm = key;
-        unsigned long long o = shfl_xor_u64(bm, 1); bm = o > bm ? o : bm;
-        o = shfl_xor_u64(bm, 8); bm = o > bm ? o : bm;
-        o = shfl_xor_u64(bm, 16); bm = o > bm ? o : bm;
-        if (m == 0 && (s & 1) == 0 && blk >= 0) bmax_row[ustep + u] = bm;
-    }
 }
 
 __device__ void stream_select_global(const unsigned long long* gk, const int* gp, int n, unsigned long long tau,
@@ -507,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
     __shared__ int kf_lut[256];
     const int K = a.plan.k;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // shared memory: staging ring | keep[2] | new   (the merge of a pool reuses the staging ring)
+    // shared memory: staging ring | keep[2] | new
     unsigned char* staging = smem;
     SelBuf B;
     {
@@ -529,10 +506,8 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
     RowCtr* rctr = reinterpret_cast<RowCtr*>(ws + a.L.row_ctr);
     unsigned long long* cand_key = reinterpret_cast<unsigned long long*>(ws + a.L.cand_key);
     int* cand_pos = reinterpret_cast<int*>(ws + a.L.cand_pos);
-    unsigned long long* bmax = reinterpret_cast<unsigned long long*>(ws + a.L.bmax);
     const int rows = a.plan.rows;
     const int total = rows * a.plan.chunks;
-    const bool pool = a.plan.pool_blocks > 0;
     unsigned char* wst = staging + warp * kStages * kStepBytes;
 
     for (;;) {
@@ -577,19 +552,18 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
                 qv[4 * i + 0] = q4.x; qv[4 * i + 1] = q4.y; qv[4 * i + 2] = q4.z; qv[4 * i + 3] = q4.w;
             }
             const int qf0 = S.qf[2 * s], qf1 = S.qf[2 * s + 1];
-            unsigned long long* bmax_row = (pool && !a.reindex) ? bmax + (size_t)row * a.plan.units_max : nullptr;
             // every warp runs the same number of steps; step i of warp w covers units
             // u0 + 32 i + 4 w .. +3; a selection flush follows every kStepsPerFlush steps
             const int nsteps = (u1 - u0 + kWarps * kUnitsPerStep - 1) / (kWarps * kUnitsPerStep);
             static_assert(kStages == 2, "two staging slots");
-            int pk0 = stage_step(a, R, u0 + kUnitsPerStep * warp, u1, wst, status), pk1 = -16;
+            int pk0 = stage_step(a, R, u0 + kUnitsPerStep * warp, u1, wst), pk1 = -16;
             cp_async_commit();
             unsigned long long thr = S.thr;
             for (int i = 0; i < nsteps; ++i) {
                 const int nx = i + 1;
                 if (nx < nsteps) {
                     const int p = stage_step(a, R, u0 + kWarps * kUnitsPerStep * nx + kUnitsPerStep * warp, u1,
-                                             wst + (nx & 1) * kStepBytes, status);
+                                             wst + (nx & 1) * kStepBytes);
                     if (nx & 1) pk1 = p; else pk0 = p;
                 }
                 cp_async_commit();
@@ -597,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
                 __syncwarp();
                 score_step<RELU>(wst + (i & 1) * kStepBytes, (i & 1) ? pk1 : pk0,
                                  u0 + kWarps * kUnitsPerStep * i + kUnitsPerStep * warp, qv, qf0, qf1, kf_lut, B, S,
-                                 thr, bmax_row);
+                                 thr);
                 __syncwarp();
                 if ((i + 1) % kStepsPerFlush == 0 || i + 1 == nsteps) {
                     __syncthreads();
@@ -665,27 +639,6 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
             for (int i = tid; i < K; i += kThreads) out[i] = i < n ? buf[i] : -1;
             __syncthreads();
         }
-        if (pool && !a.reindex) {
-            const int P = a.plan.pool_blocks;
-            SelBuf PB;  // the staging ring is idle during a merge: pool buffers live there
-            unsigned char* p = staging;
-            PB.keep_key[0] = reinterpret_cast<unsigned long long*>(p); p += 8 * P;
-            PB.keep_key[1] = reinterpret_cast<unsigned long long*>(p); p += 8 * P;
-            PB.keep_pos[0] = reinterpret_cast<int*>(p); p += 4 * P;
-            PB.keep_pos[1] = reinterpret_cast<int*>(p);
-            PB.new_key = B.new_key;
-            PB.new_pos = B.new_pos;
-            stream_select_global(bmax + (size_t)row * a.plan.units_max, nullptr, R.n_units, 0ull, P, PB, hist, S, true);
-            const int n = S.nkeep, c = S.cur;
-            int* buf = reinterpret_cast<int*>(PB.keep_key[c ^ 1]);
-            for (int i = tid; i < n; i += kThreads) buf[i] = PB.keep_pos[c][i];
-            __syncthreads();
-            sort_ascending(buf, n);
-            int32_t* outp = a.out_pool + (size_t)R.b * P;
-            for (int i = tid; i < P; i += kThreads) outp[i] = i < n ? buf[i] : -1;
-            if (tid == 0) a.out_pool_n[R.b] = n;
-            __syncthreads();
-        }
         if (tid == 0) { rc->ticket = 0; rc->ncand = 0; rc->tau = 0; }
         __syncthreads();
     }
@@ -706,6 +659,8 @@ size_t smem_bytes(const IndexPlan& p) {
 }  // namespace
 
 cudaError_t launch_index(const IndexArgs& a, cudaStream_t s) {
+    // rows of one query per sequence (Full with a pool, Reindex) take index_decode.cu
+    if (a.reindex || a.plan.pool_blocks > 0) return cudaErrorInvalidValue;
     const size_t smem = smem_bytes(a.plan);
     const bool relu = (a.flags & CSA2_SCORE_RELU) != 0;
     const void* fn = relu ? (const void*)index_kernel<true> : (const void*)index_kernel<false>;
