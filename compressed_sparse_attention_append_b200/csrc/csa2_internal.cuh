@@ -134,10 +134,10 @@ struct IndexPlan {
     int rows;          // batch * tq
     int k;
     int units_max;     // 8-position units scanned per row (upper bound)
-    int chunk_units;   // units per work item
-    int chunks;        // work items per row
+    int chunk_units;   // units per work item (several-row plans)
+    int chunks;        // work items per row (several-row plans)
     int pool_blocks;   // 0 = no pool
-    size_t cand_cap;   // candidate slots per row
+    size_t cand_cap;   // candidate slots per row (decode rows: one key per position)
     int decode;        // 1: one query row per sequence, scored by score_kernel then select_kernel
 };
 
@@ -189,16 +189,9 @@ inline IndexPlan make_index_plan(int rows, int tq, int k, int64_t max_scan, int 
     p.units_max = (int)((max_scan + kBS - 1) / kBS);
     if (p.units_max < 1) p.units_max = 1;
     if (tq == 1) {
-        // decode rows: every position's key is stored (8 bytes against 144 bytes of indexer entry),
-        // work items of chunk_units units sized for about 4 items per resident warp (148 SMs x 16)
+        // decode rows: one orderable key per position (8 bytes against 144 bytes of indexer entry),
+        // plus the select kernel's histograms and candidate lists (make_layout)
         p.decode = 1;
-        const long long units = (long long)rows * p.units_max;
-        long long cu = (units + 148 * 16 * 4 - 1) / (148 * 16 * 4);
-        cu = (cu + 3) / 4 * 4;
-        if (cu < 16) cu = 16;
-        if (cu > 512) cu = 512;
-        p.chunk_units = (int)cu;
-        p.chunks = (p.units_max + p.chunk_units - 1) / p.chunk_units;
         p.cand_cap = (size_t)p.units_max * kBS;
         return p;
     }

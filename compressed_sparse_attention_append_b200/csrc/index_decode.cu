@@ -1,10 +1,12 @@
-// index_decode.cu -- the index step for decode rows (one query row per sequence) in two kernels.
+// index_decode.cu -- the index step for decode rows (one query row per sequence): zero_kernel,
+// score_kernel, select_kernel.
 //
 // Same method and the same exact integer scores as index.cu (see its header): [B] "DeepSeek Cuts
 // KV Cache Footprint Fourfold", "Technical Approach" (Full / Reindex selection); [C] "DeepSeek-V4.1-
 // Flash: Pushing KV Cache Compression to 890 Bytes per Token", sec. VI "Shortlist-of-a-shortlist"
 // and sec. IX Figure 4 (block pool), sec. XI (FP4 indexer queries and keys).
 //
+// zero_kernel: clears the rows' score histograms.
 // score_kernel: CTAs of 8 independent warps, two per SM. The rows' steps of 4 units (32 positions)
 //   are laid end to end and split evenly over all resident warps; each warp streams its steps
 //   through a private 3-stage cp.async ring. Lane l scores step position l on its own (all 256
@@ -12,11 +14,13 @@
 //   so no cross-lane sum is needed. It writes one orderable 64-bit key per position (0 for a
 //   position that is not visible), counts each key into the row's histogram by key_bin, and for a
 //   Full pool writes (and counts) the maximum key of each unit. No block-wide synchronisation.
-// select_kernel: one CTA per row. The row's histogram gives the bin that holds its k-th largest
-//   key; one pass over the keys compacts those in that bin or above into shared memory; the keys
-//   above it are taken and the keys in it ranked exactly (ties to the lower position). The selected
-//   positions come out ascending. Then the pool (top blocks by maximum key, ties to the lower
-//   block id) the same way. Rows the histogram cannot settle fall back to an exact radix select.
+// select_kernel: rows x slices of CTAs, one resident wave. The row's histogram gives the bin that
+//   holds its k-th largest key; every CTA appends its keys in that bin or above to the row's
+//   candidate list (and counts the cut-bin keys into a second-level histogram); the last CTA of
+//   the row takes the keys above the cut, ranks the few keys left at the second-level cut exactly
+//   (ties to the lower position), and writes the positions in ascending order. Then the pool (top
+//   blocks by maximum key, ties to the lower block id) the same way. Rows the histograms cannot
+//   settle fall back to an exact radix select over all of the row's keys.
 #include "csa2_internal.cuh"
 
 namespace csa2 {
@@ -650,37 +654,6 @@ __device__ int cut_bin(const unsigned int* h, int nbins, int K, SelScal& S, int*
     const int d = S.digit;
     __syncthreads();
     return d;
-}
-
-// Appends the flagged (key, element << 32 | position) pairs of the CTA to a row's candidate list:
-// one atomic per warp on the row's counter. At most kSelCand are stored; the counter keeps the count.
-template <int N>
-__device__ __forceinline__ void append_cands(const bool (&take)[N], const unsigned long long (&key)[N],
-                                             const unsigned long long (&ip)[N], unsigned int* counter,
-                                             unsigned long long* ck, unsigned long long* cip) {
-    const int lane = threadIdx.x & 31;
-    int cnt = 0;
-#pragma unroll
-    for (int j = 0; j < N; ++j) cnt += take[j];
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-    }
-    const int wtotal = __shfl_sync(0xffffffffu, incl, 31);
-    if (wtotal == 0) return;
-    int base = 0;
-    if (lane == 31) base = (int)atomicAdd(counter, (unsigned)wtotal);
-    base = __shfl_sync(0xffffffffu, base, 31);
-    int o = base + incl - cnt;
-#pragma unroll
-    for (int j = 0; j < N; ++j) {
-        if (take[j]) {
-            if (o < kSelCand) { ck[o] = key[j]; cip[o] = ip[j]; }
-            ++o;
-        }
-    }
 }
 
 // Warp-aggregated append of (element, position) to the selected list (at most K kept).

@@ -56,9 +56,11 @@ def test_full_mode_matches_oracle(orc, B, n, k, pool, sigma, ragged):
             assert np.array_equal(out[b].cpu().numpy(), ridx), (rep, b)
 
 
-def test_full_mode_multi_row_queries(orc):
-    """tq > 1 query rows per sequence (the prefill form): every row ranks its own visible prefix."""
-    B, n, tq, k = 2, 5000, 3, 256
+@pytest.mark.parametrize("tq", [3, 5])
+def test_full_mode_multi_row_queries(orc, tq):
+    """tq > 1 query rows per sequence (the prefill form, and 5 draft positions verified together):
+    every row ranks its own visible prefix."""
+    B, n, k = 2, 5000, 256
     seed = 91
     shape, cache, swa_cap = _setup(B, n, seed)
     qpos = [[n - 1 - 700 * b - 13 * t for t in range(tq)] for b in range(B)]
