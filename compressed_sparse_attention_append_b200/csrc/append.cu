@@ -71,6 +71,8 @@ __device__ __forceinline__ void quantize_block(const float (&x)[16], uint2& code
 }
 
 __global__ void __launch_bounds__(192) append_kernel(AppendArgs a) {
+    // the slots written here may still be read by the previous step's attention (the window ring)
+    wait_prior_grid();
     const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const long long ntok = (long long)a.batch * a.t;
     if (id >= ntok * 48) return;
@@ -127,8 +129,7 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
     if (threads == 0) return cudaSuccess;
     const int blk = 192;
     const long long grid = (threads + blk - 1) / blk;
-    append_kernel<<<(unsigned)grid, blk, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_after_prior(append_kernel, dim3((unsigned)grid), dim3(blk), 0, s, a);
 }
 
 }  // namespace csa2

@@ -7,6 +7,8 @@
 // and sec. IX Figure 4 (block pool), sec. XI (FP4 indexer queries and keys).
 //
 // zero_kernel: clears the rows' score histograms.
+// Every kernel here launches with programmatic stream serialisation and waits for the kernel
+// before it (griddepcontrol.wait) before touching memory that kernel may use.
 // score_kernel: CTAs of 8 independent warps, two per SM. The rows' steps of 4 units (32 positions)
 //   are laid end to end and split evenly over all resident warps; each warp streams its steps
 //   through a private 3-stage cp.async ring. Lane l scores step position l on its own (all 256
@@ -950,6 +952,7 @@ __global__ void __launch_bounds__(kQThreads, 8) select_kernel(IndexArgs a, int s
 }
 
 __global__ void zero_kernel(uint4* p, size_t n16) {
+    wait_prior_grid();  // the previous select may still read these histograms
     for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
         p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
@@ -964,9 +967,8 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s) {
     const size_t smem = (size_t)kSWarps * kWarpBytes;
     // the score histograms start from zero (kRowHist * 4 bytes per row: a multiple of 16)
     const size_t n16 = (size_t)a.plan.rows * kRowHist / 4;
-    zero_kernel<<<(unsigned)((n16 + 1023) / 1024 < 1184 ? (n16 + 1023) / 1024 : 1184), 256, 0, s>>>(
-        reinterpret_cast<uint4*>(a.ws + a.L.key_hist), n16);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_after_prior(zero_kernel, dim3((unsigned)((n16 + 1023) / 1024 < 1184 ? (n16 + 1023) / 1024 : 1184)),
+                                       dim3(256), 0, s, reinterpret_cast<uint4*>(a.ws + a.L.key_hist), n16);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

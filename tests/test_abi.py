@@ -69,6 +69,25 @@ def test_workspace_size_is_monotone_and_validates(L):
     assert e.value.status == csa.CSA2_ERR_INVALID_ARG
 
 
+def test_decode_workspace_covers_every_region(L):
+    """A decode-row workspace must hold, per row: one 8-byte key per scanned position, the score
+    histograms (2 x 2048 + 2 x 1024 four-byte bins), two candidate lists of 4096 (key, position)
+    pairs, and with a pool the block maxima (rows of an even number of 8-byte entries); plus the
+    fixed counter area (status header, 65,536 row counters of 16 bytes, 65,536 attention tickets).
+    A multi-row (prefill) plan needs none of the decode regions."""
+    sh = csa.make_shape()
+    fixed = 256 + 16 * 65536 + 4 * 65536
+    for rows, scan, pool in ((1, 4096, 0), (128, 16000, 0), (64, 131072, 2048), (3, 1000, 125)):
+        units = (scan + 7) // 8
+        bmax = ((units + 1) // 2 * 2) * 8 if pool else 0
+        need = fixed + rows * (units * 8 * 8 + (2 * 2048 + 2 * 1024) * 4 + 2 * 4096 * 16 + bmax)
+        got = csa.csa2_workspace_size(sh, rows, 1, 512, scan, pool)
+        assert got >= need, (rows, scan, pool, got, need)
+        assert got < need + 16 * 256 + rows * 16 * 132 * 4 * 64  # alignment and attention partials only
+    # the same rows as 4 prefill rows each: no per-position keys, only candidate slots
+    assert csa.csa2_workspace_size(sh, 8, 4, 512, 4096) < csa.csa2_workspace_size(sh, 32, 1, 512, 4096)
+
+
 def _fake_cache(cap=4096, swa_cap=128, align=16):
     base = 1 << 40
     return csa.csa2_cache(base, base + 1 * align * 1024, base + 2 * align * 1024, base + 3 * align * 1024,
