@@ -72,9 +72,9 @@ def lib():
             "orc_scores": (None, [vp, vp, i, vp, i64, i, vp]),
             "orc_topk": (i, [vp, vp, i64, i, vp]),
             "orc_pool": (i, [vp, i64, i, i, vp]),
-            "orc_index_topk_full": (i, [vp, i64, vp, i, i, i, vp, i, i, vp, vp]),
-            "orc_index_topk_reindex": (i, [vp, i64, vp, i, vp, i, i, i, i, vp]),
-            "orc_sparse_attend": (i, [vp, i64, vp, i, vp, i, i64, i, d, vp, vp]),
+            "orc_index_topk_full": (i, [vp, i64, vp, i, i, i, vp, i, i, vp, vp, i]),
+            "orc_index_topk_reindex": (i, [vp, i64, vp, i, vp, i, i, i, i, vp, i]),
+            "orc_sparse_attend": (i, [vp, i64, vp, i, vp, i, i64, i, d, vp, vp, i]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -216,27 +216,33 @@ class SeqCache:
         lib().orc_scores(self.ref, _p(q), q.size // 64, _p(p), p.size, 1, _p(out))
         return out
 
-    def index_topk_full(self, qpos: int, idx_q, k: int = 512, pool_blocks: int = 0, bs: int = 8, relu=False):
+    def index_topk_full(self, qpos: int, idx_q, k: int = 512, pool_blocks: int = 0, bs: int = 8, relu=False,
+                        ratio: int = 1):
+        """Full mode at token qpos; with compression ratio `ratio` the first (qpos + 1) // ratio
+        entries are visible (R12)."""
         q = _bf16_bits(idx_q).reshape(-1)
         out = np.zeros(k, np.int32)
         pool_out = np.zeros(max(pool_blocks, 1), np.int32)
         pool_n = np.zeros(1, np.int32)
         lib().orc_index_topk_full(self.ref, qpos, _p(q), q.size // 64, k, int(relu), _p(out),
-                                  pool_blocks, bs, _p(pool_out), _p(pool_n))
+                                  pool_blocks, bs, _p(pool_out), _p(pool_n), int(ratio))
         if pool_blocks > 0:
             return out, pool_out, int(pool_n[0])
         return out
 
-    def index_topk_reindex(self, qpos: int, idx_q, pool_ids, pool_n: int, k: int = 512, bs: int = 8, relu=False):
+    def index_topk_reindex(self, qpos: int, idx_q, pool_ids, pool_n: int, k: int = 512, bs: int = 8, relu=False,
+                           ratio: int = 1):
         q = _bf16_bits(idx_q).reshape(-1)
         pl = np.ascontiguousarray(pool_ids, np.int32)
         out = np.zeros(k, np.int32)
         lib().orc_index_topk_reindex(self.ref, qpos, _p(q), q.size // 64, _p(pl), int(pool_n), bs, k,
-                                     int(relu), _p(out))
+                                     int(relu), _p(out), int(ratio))
         return out
 
-    def sparse_attend(self, qpos: int, q, idx, swa_begin: int = 0, win: int = 128, sm_scale: float = 0.0):
-        """R7/R8: one softmax over selected FP4 rows and the FP8 window; fp64 out [hq,128], lse [hq]."""
+    def sparse_attend(self, qpos: int, q, idx, swa_begin: int = 0, win: int = 128, sm_scale: float = 0.0,
+                      ratio: int = 1):
+        """R7/R8: one softmax over selected FP4 rows and the FP8 window; fp64 out [hq,128], lse [hq].
+        Selected entries must be visible at token qpos (R12); the window is per token."""
         qb = _bf16_bits(q).reshape(-1)
         hq = qb.size // 128
         ix = np.ascontiguousarray(idx, np.int32).reshape(-1)
@@ -245,7 +251,7 @@ class SeqCache:
         out = np.zeros((hq, 128), np.float64)
         lse = np.zeros(hq, np.float64)
         nk = lib().orc_sparse_attend(self.ref, qpos, _p(qb), hq, _p(ix), ix.size, swa_begin, win,
-                                     float(sm_scale), _p(out), _p(lse))
+                                     float(sm_scale), _p(out), _p(lse), int(ratio))
         if nk < 0:
             raise ValueError("index out of range")
         return out, lse

@@ -37,7 +37,9 @@
  *       covers positions 8b .. 8b+7.
  *   R11 a decode query sits at N - 1 and is appended before scoring (so it is visible);
  *       prefill row i sees positions <= i.
- *   R12 compression ratio 1: one cache entry per token.
+ *   R12 compression ratio r in {1, 2}: cache entry e summarises tokens r*e .. r*e + r - 1 and is
+ *       visible to a query at token i once all of them are <= i, i.e. the first floor((i + 1) / r)
+ *       entries; the window stays per token.
  *
  * Parity pins: every function here is checked by tests/test_oracle_*.py against exact
  * rational arithmetic, library routines (torch float8 conversion, Python sorted(), torch
@@ -320,14 +322,18 @@ ORC_API int orc_pool(const double* scores, int64_t n, int bs, int pool_blocks, i
     return m;
 }
 
-/* Full mode index step for one query at position qpos (R11: positions 0..qpos visible).
- * [B] "Technical Approach"; [C] sec. VI "Shortlist-of-a-shortlist": scores every causally
- * visible position, keeps Top-k, and (pool_blocks > 0) builds the block pool. */
+/* Entries visible to a query at token qpos (R11, R12): entry e covers tokens ratio*e ..
+ * ratio*e + ratio - 1, all of which must be <= qpos. */
+static int64_t orc_visible(int64_t qpos, int ratio) { return qpos < 0 ? 0 : (qpos + 1) / ratio; }
+
+/* Full mode index step for one query at token qpos (R11, R12: the visible entries are 0 ..
+ * orc_visible - 1). [B] "Technical Approach"; [C] sec. VI "Shortlist-of-a-shortlist": scores
+ * every causally visible entry, keeps Top-k, and (pool_blocks > 0) builds the block pool. */
 ORC_API int orc_index_topk_full(const orc_seq_cache* c, int64_t qpos, const uint16_t* idx_q, int hi, int k,
                                 int relu, int32_t* out_idx, int pool_blocks, int bs, int32_t* out_pool,
-                                int32_t* out_pool_n)
+                                int32_t* out_pool_n, int ratio)
 {
-    int64_t n = qpos + 1;
+    int64_t n = orc_visible(qpos, ratio);
     int64_t* p = (int64_t*)malloc(sizeof(int64_t) * n);
     double* s = (double*)malloc(sizeof(double) * n);
     for (int64_t i = 0; i < n; ++i) p[i] = i;
@@ -339,17 +345,19 @@ ORC_API int orc_index_topk_full(const orc_seq_cache* c, int64_t qpos, const uint
 }
 
 /* Reindex mode: [B] "Technical Approach" and [C] sec. VI: a fresh indexer query picks its
- * Top-k only among the pool's positions {bs*b .. bs*b+bs-1 : b in pool}, limited to
- * positions <= qpos. */
+ * Top-k only among the pool's positions {bs*b .. bs*b+bs-1 : b in pool}, limited to the
+ * entries visible at token qpos (R12). */
 ORC_API int orc_index_topk_reindex(const orc_seq_cache* c, int64_t qpos, const uint16_t* idx_q, int hi,
-                                   const int32_t* pool, int pool_n, int bs, int k, int relu, int32_t* out_idx)
+                                   const int32_t* pool, int pool_n, int bs, int k, int relu, int32_t* out_idx,
+                                   int ratio)
 {
+    const int64_t vis = orc_visible(qpos, ratio);
     int64_t* p = (int64_t*)malloc(sizeof(int64_t) * ((int64_t)pool_n * bs + 1));
     int64_t n = 0;
     for (int i = 0; i < pool_n; ++i)
         for (int j = 0; j < bs; ++j) {
             int64_t q = (int64_t)pool[i] * bs + j;
-            if (q <= qpos) p[n++] = q;
+            if (q < vis) p[n++] = q;
         }
     double* s = (double*)malloc(sizeof(double) * (n + 1));
     orc_scores(c, idx_q, hi, p, n, relu, s);
@@ -367,8 +375,9 @@ ORC_API int orc_index_topk_reindex(const orc_seq_cache* c, int64_t qpos, const u
 /* ------------------------------------------------------------------------------------ */
 ORC_API int orc_sparse_attend(const orc_seq_cache* c, int64_t qpos, const uint16_t* q /*[hq][128]*/, int hq,
                               const int32_t* idx, int k, int64_t swa_begin, int win, double sm_scale,
-                              double* out /*[hq][128]*/, double* lse /*[hq]*/)
+                              double* out /*[hq][128]*/, double* lse /*[hq]*/, int ratio)
 {
+    const int64_t vis = orc_visible(qpos, ratio);  /* selected entries must be visible (R12) */
     int64_t lo = qpos - win + 1;
     if (lo < swa_begin) lo = swa_begin;
     if (lo < 0) lo = 0;
@@ -380,7 +389,7 @@ ORC_API int orc_sparse_attend(const orc_seq_cache* c, int64_t qpos, const uint16
     double row[256];
     for (int j = 0; j < k; ++j) {
         if (idx[j] < 0) continue;
-        if (idx[j] > qpos || idx[j] >= c->cap) { free(K); free(V); return -1; }
+        if (idx[j] >= vis || idx[j] >= c->cap) { free(K); free(V); return -1; }
         orc_dequant_rows(c->kv_data + (int64_t)idx[j] * 128, c->kv_scale + (int64_t)idx[j] * 16, 1, 256, row);
         memcpy(K + nk * 128, row, 128 * sizeof(double));
         memcpy(V + nk * 128, row + 128, 128 * sizeof(double));

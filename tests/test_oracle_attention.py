@@ -122,3 +122,18 @@ def test_default_scale_is_inverse_sqrt_d(orc):
     a, la = c.sparse_attend(19, q, idx, sm_scale=0.0)
     b, lb = c.sparse_attend(19, q, idx, sm_scale=1 / np.sqrt(128))
     assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_ratio_two_selected_rows_must_be_complete(orc):
+    """R12 with r = 2: a query at token 150 may use entries 0..74 (entry 74 covers tokens 148, 149);
+    entry 75 covers token 151, which is in the future. The window stays per token."""
+    c, q = build(orc, 200, seed=12)
+    qpos, scale = 150, 1.0 / np.sqrt(128.0)
+    idx = np.array([0, 10, 74, -1], np.int32)
+    out, lse = c.sparse_attend(qpos, q, idx, ratio=2)
+    want, wl = dense(c, q, [0, 10, 74], list(range(qpos - 127, qpos + 1)), scale)
+    np.testing.assert_allclose(out, want, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, wl, rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        c.sparse_attend(qpos, q, np.array([75], np.int32), ratio=2)
+    c.sparse_attend(qpos, q, np.array([75], np.int32), ratio=1)  # visible without compression

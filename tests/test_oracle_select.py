@@ -154,3 +154,29 @@ def test_full_mode_small_context(orc):
     q = torch.randn(4, 64, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
     idx = c.index_topk_full(9, q, k=16)
     assert idx.tolist() == list(range(10)) + [-1] * 6
+
+
+@pytest.mark.parametrize("qpos", [0, 1, 2, 3, 98, 99, 150, 201])
+def test_ratio_two_sees_only_complete_entries(orc, qpos):
+    """R12 with r = 2: entry e summarises tokens 2e and 2e + 1, so a query at token i may use e only
+    when 2e + 1 <= i. Full, pool and Reindex must rank exactly those entries."""
+    n = 120
+    c = make_cache(orc, n, seed=21)
+    q = torch.randn(4, 64, generator=torch.Generator().manual_seed(qpos)).to(torch.bfloat16)
+    vis = [e for e in range(n) if 2 * e + 1 <= qpos]  # brute force from the definition
+    k = 24
+    idx, pool, pool_n = c.index_topk_full(qpos, q, k=k, pool_blocks=5, ratio=2)
+    if vis:
+        s = c.scores(q, np.array(vis)).tolist()
+        assert idx.tolist() == brute_topk(s, vis, k)
+        bp, bpn = brute_pool(s, 8, 5)
+        assert pool_n == bpn and pool.tolist() == bp
+        # the same entries as the uncompressed cache queried at the last visible entry
+        assert idx.tolist() == c.index_topk_full(len(vis) - 1, q, k=k).tolist()
+    else:
+        assert idx.tolist() == [-1] * k and pool_n == 0
+    blocks = np.array([0, 4, 9, 14], np.int32)
+    got = c.index_topk_reindex(qpos, q, blocks, 4, k=k, ratio=2)
+    cand = [b * 8 + j for b in blocks for j in range(8) if b * 8 + j in set(vis)]
+    want = brute_topk(c.scores(q, np.array(cand)).tolist(), cand, k) if cand else [-1] * k
+    assert got.tolist() == want
