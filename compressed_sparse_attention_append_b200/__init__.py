@@ -45,7 +45,7 @@ class Csa2Error(RuntimeError):
 
 
 class csa2_shape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int) for n in ("hq", "d", "hi", "di", "hk", "win", "bs")]
+    _fields_ = [(n, ctypes.c_int) for n in ("hq", "d", "hi", "di", "hk", "win", "bs", "ratio")]
 
 
 class csa2_cache(ctypes.Structure):
@@ -124,8 +124,8 @@ def _stream(stream):
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def make_shape(win: int = 128) -> csa2_shape:
-    return csa2_shape(hq=16, d=128, hi=4, di=64, hk=4, win=win, bs=8)
+def make_shape(win: int = 128, ratio: int = 1) -> csa2_shape:
+    return csa2_shape(hq=16, d=128, hi=4, di=64, hk=4, win=win, bs=8, ratio=ratio)
 
 
 class Cache:

@@ -15,7 +15,7 @@ bool al16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 csa2_status check_shape(const csa2_shape* s) {
     if (!s) return CSA2_ERR_INVALID_ARG;
     if (s->hq != kHQ || s->d != kD || s->hi != kHI || s->di != kDI || s->hk != kHK || s->bs != kBS ||
-        s->win < 0 || s->win > 128)
+        s->win < 0 || s->win > 128 || (s->ratio != 1 && s->ratio != 2))
         return CSA2_ERR_UNSUPPORTED_SHAPE;
     return CSA2_OK;
 }
@@ -109,6 +109,7 @@ csa2_status do_index(const csa2_shape* shape, const csa2_cache* cache, int batch
     a.pool_n = pool_n;
     a.pool_stride = pool_stride;
     a.max_ctx = reindex ? cache->cap : max_ctx;
+    a.ratio = shape->ratio;
     a.out_idx = out_idx;
     a.out_pool = out_pool;
     a.out_pool_n = out_pool_n;
@@ -141,6 +142,7 @@ csa2_status do_attend(const csa2_shape* shape, const csa2_cache* cache, int batc
     a.tq = tq;
     a.k = k;
     a.win = shape->win;
+    a.ratio = shape->ratio;
     a.qpos = qpos;
     a.qpos_base = qpos_base;
     a.swa_begin_host = swa_begin_host;
@@ -179,7 +181,7 @@ const char* csa2_status_string(csa2_status s) {
     return "unknown status";
 }
 
-int csa2_version(void) { return 100; }
+int csa2_version(void) { return 101; }
 
 csa2_status csa2_workspace_size(const csa2_shape* shape, int batch, int tq, int k, int64_t max_scan, int pool_blocks,
                                 size_t* bytes) {
@@ -239,6 +241,8 @@ csa2_status csa2_decode_full(const csa2_shape* shape, const csa2_cache* cache, i
                              uint16_t* out, float* out_f32, float* lse, uint32_t flags, void* ws, size_t ws_bytes,
                              void* stream) {
     if (!qpos || !kv || !idx_k || !swa_kv) return CSA2_ERR_INVALID_ARG;
+    CSA2_TRY(check_shape(shape));
+    if (shape->ratio != 1) return CSA2_ERR_UNSUPPORTED_SHAPE;  // an entry per token only
     CSA2_TRY(do_append(shape, cache, batch, 1, qpos, 0, kv, idx_k, swa_kv, ws, ws_bytes, stream));
     CSA2_TRY(do_index(shape, cache, batch, 1, qpos, 0, idx_q, k, out_idx, pool_blocks, out_pool, out_pool_n, max_ctx, 0,
                       nullptr, nullptr, 0, flags, ws, ws_bytes, stream));
@@ -275,6 +279,8 @@ csa2_status csa2_prefill_chunk(const csa2_shape* shape, const csa2_cache* cache,
                                float sm_scale, uint16_t* out, float* out_f32, float* lse, uint32_t flags, void* ws,
                                size_t ws_bytes, void* stream) {
     if (!shape || !cache || !kv || !idx_k || !swa_kv || t < 1 || pos0 < 0) return CSA2_ERR_INVALID_ARG;
+    CSA2_TRY(check_shape(shape));
+    if (shape->ratio != 1) return CSA2_ERR_UNSUPPORTED_SHAPE;  // an entry per token only
     if (pos0 + t > cache->cap) return CSA2_ERR_CAPACITY;
     if (cache->swa_cap < (int64_t)t + (shape ? shape->win : 0)) return CSA2_ERR_CAPACITY;
     CSA2_TRY(do_append(shape, cache, 1, t, nullptr, pos0, kv, idx_k, swa_kv, ws, ws_bytes, stream));

@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
     RowKeys R;
     R.b = row / a.tq;
     R.qpos = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
-    const bool row_ok = R.qpos >= 0 && R.qpos < a.c.cap;
+    const int64_t qlast = R.qpos < 0 ? -1 : (R.qpos + 1) / a.ratio - 1;  // the last visible entry
+    const bool row_ok = R.qpos >= 0 && qlast < a.c.cap;
     // ---- Q -> fp16 in shared memory (thread: head tid>>4, dims 8*(tid&15) .. +7) ----
     {
         const int h = tid >> 4, c = tid & 15;
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
     for (int r = 0; r < rounds; ++r) {
         const int i = r * kAThreads + tid;
         const int v = i < K ? idx[i] : -1;
-        const bool ok = row_ok && v >= 0 && v <= R.qpos && (int64_t)v < a.c.cap;
+        const bool ok = row_ok && v >= 0 && v <= qlast && (int64_t)v < a.c.cap;
         if (!ok && v != -1 && split == 0) set_status(status, CSA2_DEV_BAD_INDEX);
         const unsigned int bal = __ballot_sync(0xffffffffu, ok);
         if (lane == 0) s_cnt[r * kAWarps + warp] = __popc(bal);
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attend_kernel(AttendArgs a) {
     for (int r = 0; r < rounds; ++r) {
         const int i = r * kAThreads + tid;
         const int v = i < K ? idx[i] : -1;
-        const bool ok = row_ok && v >= 0 && v <= R.qpos && (int64_t)v < a.c.cap;
+        const bool ok = row_ok && v >= 0 && v <= qlast && (int64_t)v < a.c.cap;
         const unsigned int bal = __ballot_sync(0xffffffffu, ok);
         if (ok) list[s_cnt[r * kAWarps + warp] + __popc(bal & ((1u << lane) - 1))] = v;
     }

@@ -270,7 +270,8 @@ struct IndexArgs {
     const int32_t* pool; // Reindex: [batch][pool_stride]
     const int32_t* pool_n;
     int pool_stride;
-    int64_t max_ctx;     // Full: bound on qpos+1
+    int64_t max_ctx;     // Full: bound on the visible entries
+    int ratio;           // tokens per cache entry (1 or 2): a row at token q sees (q + 1) / ratio entries
     int32_t* out_idx;
     int32_t* out_pool;
     int32_t* out_pool_n;
@@ -285,6 +286,7 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s);  // index_d
 struct AttendArgs {
     csa2_cache c;
     int rows, tq, k, win;
+    int ratio;            // tokens per cache entry: selected entries must be < (qpos + 1) / ratio
     const int64_t* qpos;  // or NULL: qpos_base + r % tq
     int64_t qpos_base;
     int64_t swa_begin_host;  // used when swa_begin is NULL

@@ -348,9 +348,10 @@ struct RowInfo {
 __device__ RowInfo row_info(const IndexArgs& a, int row) {
     RowInfo r;
     r.b = row / a.tq;
-    r.qpos = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
+    const int64_t tok = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
+    r.qpos = tok < 0 ? -1 : (tok + 1) / a.ratio - 1;  // the last visible entry
     r.ok = true;
-    if (r.qpos < 0 || r.qpos >= a.c.cap || r.qpos >= a.max_ctx) {
+    if (tok < 0 || r.qpos >= a.c.cap || r.qpos >= a.max_ctx) {
         r.ok = false;
         r.n_units = 0;
         return r;

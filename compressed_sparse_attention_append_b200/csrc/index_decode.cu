@@ -98,7 +98,7 @@ __device__ __forceinline__ int sub_bin(unsigned long long key) {
 }
 
 struct DRow {
-    int64_t qpos;
+    int64_t qpos;  // the last visible entry: floor((query token + 1) / ratio) - 1
     int b;
     int n_units;
 };
@@ -106,8 +106,9 @@ struct DRow {
 __device__ __forceinline__ DRow drow(const IndexArgs& a, int row, bool& ok) {
     DRow r;
     r.b = row;  // decode: tq == 1
-    r.qpos = a.qpos ? a.qpos[row] : a.qpos_base;
-    ok = !(r.qpos < 0 || r.qpos >= a.c.cap || (!a.reindex && r.qpos >= a.max_ctx));
+    const int64_t tok = a.qpos ? a.qpos[row] : a.qpos_base;
+    r.qpos = tok < 0 ? -1 : (tok + 1) / a.ratio - 1;
+    ok = !(tok < 0 || r.qpos >= a.c.cap || (!a.reindex && r.qpos >= a.max_ctx));
     if (!ok) {
         r.n_units = 0;
     } else if (a.reindex) {

@@ -57,7 +57,7 @@ extern "C" CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* sha
                                                            void* stream) {
     if (!shape || !cache) return CSA2_ERR_INVALID_ARG;
     if (shape->hq != kHQ || shape->d != kD || shape->hi != kHI || shape->di != kDI || shape->hk != kHK ||
-        shape->bs != kBS || shape->win < 0 || shape->win > 128)
+        shape->bs != kBS || shape->win < 0 || shape->win > 128 || (shape->ratio != 1 && shape->ratio != 2))
         return CSA2_ERR_UNSUPPORTED_SHAPE;
     if (cache->cap <= 0 || cache->swa_cap <= 0 || (cache->swa_cap & (cache->swa_cap - 1)) || !cache->kv_data ||
         !cache->kv_scale || !cache->swa || !al16(cache->kv_data) || !al16(cache->kv_scale) || !al16(cache->swa))
@@ -84,6 +84,7 @@ extern "C" CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* sha
     a.tq = tq;
     a.k = k;
     a.win = shape->win;
+    a.ratio = shape->ratio;
     a.qpos = qpos;
     a.q = q;
     a.idx = idx;

@@ -70,6 +70,10 @@ typedef struct {
     int hk;   /* indexer key heads (4)                            */
     int win;  /* sliding-window length (128; [C] config list)     */
     int bs;   /* positions per pool block (8; [C] sec. IX)        */
+    int ratio; /* tokens per main / indexer cache entry: 1, or 2 for the encoder layers of
+                  [C] sec. VIII (one entry per 2 tokens). Entry e summarises tokens
+                  ratio*e .. ratio*e + ratio - 1; a query at token i may use entries
+                  0 .. floor((i + 1) / ratio) - 1. Window slots stay per token. */
 } csa2_shape;
 
 /*
@@ -143,14 +147,15 @@ CSA2_API csa2_status csa2_quantize_append(const csa2_shape* shape, const csa2_ca
  * [C] sec. VI "Shortlist-of-a-shortlist" and sec. IX Figure 4: the decoder's first Full layer
  * scores every causally visible position, and collects the blocks with the highest maximum
  * score (up to 2,048 blocks of 8 positions) into a shared candidate pool.
- *   qpos     [batch*tq] int64 : query position of each row; positions 0..qpos are visible
+ *   qpos     [batch*tq] int64 : query token of each row; entries 0 .. floor((qpos+1)/ratio)-1 are
+ *              visible (with ratio 1: positions 0..qpos)
  *   idx_q    [batch][tq][hi][di] bf16 : indexer query, quantised in-kernel with the codec above
  *   k        : Top-k (<= 2048)
  *   out_idx  [batch][tq][k] int32 : selected positions, ascending, padded with -1
  *   pool_blocks : 0, or the pool size P (decode only: tq == 1)
  *   out_pool [batch][P] int32 : pool block ids, ascending, padded with -1 (NULL if P == 0)
- *   out_pool_n [batch] int32 : min(P, ceil((qpos+1)/bs))          (NULL if P == 0)
- *   max_ctx  : host upper bound on qpos+1 over all rows (<= cap)
+ *   out_pool_n [batch] int32 : min(P, ceil(visible entries / bs))  (NULL if P == 0)
+ *   max_ctx  : host upper bound on the visible entries over all rows (<= cap)
  * Score (this build's reading): score(p) = sum_h q_h . k_{p,h} on dequantised values, exact;
  * ranking by score descending, ties to the lower position (lower block id for the pool).
  */
@@ -165,7 +170,8 @@ CSA2_API csa2_status csa2_index_topk_full(const csa2_shape* shape, const csa2_ca
  *   qpos   [batch] int64, idx_q [batch][hi][di] bf16
  *   pool   [batch][pool_stride] int32 : block ids (each covers positions bs*id .. bs*id+bs-1)
  *   pool_n [batch] int32 : entries used in each row (<= pool_stride)
- *   out_idx [batch][k] int32 : ascending, padded with -1; positions > qpos are never chosen
+ *   out_idx [batch][k] int32 : ascending, padded with -1; entries that are not visible at qpos
+ *              (see ratio) are never chosen
  */
 CSA2_API csa2_status csa2_index_topk_reindex(const csa2_shape* shape, const csa2_cache* cache, int batch,
                                     const int64_t* qpos, const uint16_t* idx_q, const int32_t* pool,
@@ -177,15 +183,15 @@ CSA2_API csa2_status csa2_index_topk_reindex(const csa2_shape* shape, const csa2
  * the selected entries of the shared main KV plus its own recent window; [C] sec. XI: cached
  * values are dequantised before attention; [C] sec. XII: with a replay start s, a query at i
  * sees window keys [max(s, i-win+1), i].
- *   qpos [batch*tq] int64, q [batch][tq][hq][d] bf16
- *   idx  [batch][tq][k] int32 : main-KV positions, -1 = skip, any order
+ *   qpos [batch*tq] int64 (query token), q [batch][tq][hq][d] bf16
+ *   idx  [batch][tq][k] int32 : main-KV entries, -1 = skip, any order
  *   swa_begin [batch] int64 or NULL (= 0)
  *   sm_scale : softmax scale, 0 gives 1/sqrt(d)
  *   out [batch][tq][hq][d] bf16; out_f32 (same shape, fp32) and lse [batch][tq][hq] fp32 (natural
  *   log) may be NULL.
  * This build's reading: ONE softmax over selected rows and window rows together; a position may
  * appear in both (its FP4 main entry and its FP8 window entry are different vectors). An index
- * < -1, > qpos or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row with no key gives out = 0
+ * < -1, not visible at qpos (see ratio) or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row with no key gives out = 0
  * and lse = -inf.
  */
 CSA2_API csa2_status csa2_sparse_attend(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
@@ -200,6 +206,8 @@ CSA2_API csa2_status csa2_sparse_attend(const csa2_shape* shape, const csa2_cach
  * quantise-append -> index step -> sparse attention on `stream`, with the arguments above;
  * the new token sits at qpos[b] (appended before scoring, so it is visible).
  *   decode_full    : appends kv, idx_k, swa_kv; Full index step (pool optional); attention
+ *                    (ratio 1 only: with ratio 2 an entry is appended every second token, so the
+ *                    caller appends it and calls the index step and attention itself)
  *   decode_reindex : appends swa_kv; Reindex index step; attention
  *   decode_minimal : appends swa_kv; attention with the inherited idx
  */
@@ -228,7 +236,7 @@ CSA2_API csa2_status csa2_decode_minimal(const csa2_shape* shape, const csa2_cac
  * and XI: the chunk's K/V and indexer keys are quantised and appended; every new token then
  * selects its Top-k among positions <= its own and attends to them plus its window.
  *   kv [t][256], idx_k [t][hk*64], swa_kv [t][256], idx_q [t][hi][di], q [t][hq][d] (bf16)
- *   out_idx [t][k] int32, out [t][hq][d] bf16; swa_cap must be >= t + win.
+ *   out_idx [t][k] int32, out [t][hq][d] bf16; swa_cap must be >= t + win. ratio 1 only.
  */
 CSA2_API csa2_status csa2_prefill_chunk(const csa2_shape* shape, const csa2_cache* cache, int64_t pos0, int t,
                                const uint16_t* kv, const uint16_t* idx_k, const uint16_t* swa_kv,

@@ -47,7 +47,7 @@ def test_host_functions(L):
     assert csa.csa2_entry_bytes(256) == 144
     assert csa.csa2_entry_bytes(512) == 288
     assert csa.csa2_entry_bytes(24) == 0 and csa.csa2_entry_bytes(-16) == 0
-    assert csa.csa2_version() == 100
+    assert csa.csa2_version() == 101
     for s in range(7):
         assert csa.csa2_status_string(s)
     assert csa.csa2_status_string(99) == "unknown status"
@@ -67,6 +67,11 @@ def test_workspace_size_is_monotone_and_validates(L):
     with pytest.raises(csa.Csa2Error) as e:
         csa.csa2_workspace_size(sh, 1, 1, 4096, 4096)
     assert e.value.status == csa.CSA2_ERR_INVALID_ARG
+    # compression ratio: 1 or 2 tokens per cache entry
+    assert csa.csa2_workspace_size(csa.make_shape(ratio=2), 1, 1, 512, 4096) > 0
+    with pytest.raises(csa.Csa2Error) as e:
+        csa.csa2_workspace_size(csa.make_shape(ratio=3), 1, 1, 512, 4096)
+    assert e.value.status == csa.CSA2_ERR_UNSUPPORTED_SHAPE
 
 
 def test_decode_workspace_covers_every_region(L):
@@ -114,6 +119,12 @@ def test_validation_before_launch(L):
                                   vp, 1 << 30, None) == csa.CSA2_ERR_CAPACITY
     assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 1, 1, vp, vp, 512, vp, 0, None, None, 100, 8,
                                   vp, 1 << 30, None) == csa.CSA2_ERR_INVALID_ARG
+    # the composed decode_full and prefill_chunk calls take one entry per token only
+    r2 = csa.make_shape(ratio=2)
+    assert L.csa2_decode_full(ctypes.byref(r2), ctypes.byref(c), 1, vp, vp, vp, vp, vp, vp, 512, vp, 0, None, None,
+                              100, None, 0.0, vp, None, None, 0, vp, 1 << 30, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    assert L.csa2_prefill_chunk(ctypes.byref(r2), ctypes.byref(c), 0, 16, vp, vp, vp, vp, vp, 512, vp, 0, 0.0, vp, None,
+                                None, 0, vp, 1 << 30, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
     # workspace too small / missing
     assert L.csa2_index_topk_full(ctypes.byref(sh), ctypes.byref(c), 4, 1, vp, vp, 512, vp, 0, None, None, 4096, 0,
                                   vp, 1024, None) == csa.CSA2_ERR_WORKSPACE

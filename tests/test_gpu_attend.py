@@ -186,3 +186,35 @@ def test_prefill_chunk_matches_oracle(orc, p0, t):
         assert np.array_equal(out_idx[r].cpu().numpy(), ridx), r
         refs.append(oc.sparse_attend(p0 + r, qc[r], ridx))
     _check_rows(out[rows], of[rows], lse[rows], refs, 2e-3)
+
+
+def test_ratio_two_attention(orc):
+    """Compression ratio 2: a query at token i may use entries 0 .. floor((i + 1) / 2) - 1; the window
+    stays per token. Entry floor((i + 1) / 2) is not visible yet: flagged and skipped."""
+    B, n, k = 2, 3000, 256
+    seed = 57
+    _, cache, swa_cap = _cache(B, n, seed)
+    shape = csa.make_shape(ratio=2)
+    qpos = [2999, 2500]  # visible entries 1500 and 1250
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV)
+    q = query_values(seed, "q", torch.arange(B), qp, 2048, DEV).reshape(B, 16, 128).contiguous()
+    vis = [(p + 1) // 2 for p in qpos]
+    idx = torch.stack([W.distinct_sorted(seed, "sel", torch.tensor([b], device=DEV), vis[b], k)[0]
+                       for b in range(B)]).to(torch.int32).contiguous()
+    out = torch.empty(B, 16, 128, dtype=torch.bfloat16, device=DEV)
+    of = torch.empty(B, 16, 128, dtype=torch.float32, device=DEV)
+    lse = torch.empty(B, 16, dtype=torch.float32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, 8)
+    csa.csa2_sparse_attend(shape, cache, B, 1, qp, q, idx, k, out, out_f32=of, lse=lse, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    refs = []
+    for b in range(B):
+        oc = oracle_seq(seed, b, n, n, swa_cap)
+        qb = query_values(seed, "q", [b], [qpos[b]], 2048, "cpu")[0]
+        refs.append(oc.sparse_attend(qpos[b], qb, idx[b].cpu().numpy(), ratio=2))
+    _check_rows(out, of, lse, refs, attn_tol(None, 1.0))
+    # the first entry that is not visible yet
+    idx2 = idx.clone()
+    idx2[:, 0] = torch.tensor(vis, dtype=torch.int32, device=DEV)
+    csa.csa2_sparse_attend(shape, cache, B, 1, qp, q, idx2, k, out, out_f32=of, lse=lse, ws=ws)
+    assert csa.csa2_get_device_status(ws) == csa.CSA2_DEV_BAD_INDEX

@@ -56,13 +56,14 @@ def test_full_mode_matches_oracle(orc, B, n, k, pool, sigma, ragged):
             assert np.array_equal(out[b].cpu().numpy(), ridx), (rep, b)
 
 
-@pytest.mark.parametrize("tq", [3, 5])
-def test_full_mode_multi_row_queries(orc, tq):
+@pytest.mark.parametrize("tq,ratio", [(3, 1), (5, 1), (3, 2)])
+def test_full_mode_multi_row_queries(orc, tq, ratio):
     """tq > 1 query rows per sequence (the prefill form, and 5 draft positions verified together):
-    every row ranks its own visible prefix."""
+    every row ranks its own visible prefix (with ratio 2: the entries whose two tokens precede it)."""
     B, n, k = 2, 5000, 256
     seed = 91
-    shape, cache, swa_cap = _setup(B, n, seed)
+    _, cache, swa_cap = _setup(B, n, seed)
+    shape = csa.make_shape(ratio=ratio)
     qpos = [[n - 1 - 700 * b - 13 * t for t in range(tq)] for b in range(B)]
     qp = torch.tensor(qpos, dtype=torch.int64, device=DEV).reshape(-1)
     rows_b = torch.arange(B).repeat_interleave(tq)
@@ -75,7 +76,7 @@ def test_full_mode_multi_row_queries(orc, tq):
         oc = oracle_seq(seed, b, n, n, swa_cap)
         for t in range(tq):
             qb = query_values(seed, "iq", [b], [qpos[b][t]], 256, "cpu")[0]
-            ref = oc.index_topk_full(qpos[b][t], qb, k=k)
+            ref = oc.index_topk_full(qpos[b][t], qb, k=k, ratio=ratio)
             assert np.array_equal(out[b * tq + t].cpu().numpy(), ref), (b, t)
 
 
@@ -238,3 +239,36 @@ def test_bad_pool_id_sets_status():
     assert csa.csa2_get_device_status(ws) == csa.CSA2_DEV_BAD_POOL
     got = out[0].cpu().numpy()
     assert set(got[got >= 0].tolist()) == set(range(0, 8)) | set(range(24, 32))
+
+
+def test_ratio_two_full_and_reindex(orc):
+    """Compression ratio 2: the rows at tokens 2n - 1 and 2n - 6 see the first n and n - 3 entries
+    (entry e summarises tokens 2e, 2e + 1). Full (with its pool) and Reindex against the oracle."""
+    B, n, k, P = 2, 6000, 256, 300
+    seed = 63
+    _, cache, swa_cap = _setup(B, n, seed)
+    shape = csa.make_shape(ratio=2)
+    qpos = [2 * n - 1, 2 * n - 6]
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV)
+    iq = query_values(seed, "iq", torch.arange(B), qp, 256, DEV).contiguous()
+    out = torch.empty(B, k, dtype=torch.int32, device=DEV)
+    opool = torch.empty(B, P, dtype=torch.int32, device=DEV)
+    opn = torch.empty(B, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, 1, k, n, P)
+    csa.csa2_index_topk_full(shape, cache, B, 1, qp, iq, k, out, P, opool, opn, max_ctx=n, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    pool = W.distinct_sorted(seed, "pool", torch.arange(B, device=DEV), n // 8, 400).to(torch.int32).contiguous()
+    pool_n = torch.tensor([400, 390], dtype=torch.int32, device=DEV)
+    out2 = torch.empty(B, k, dtype=torch.int32, device=DEV)
+    ws2 = csa.Workspace(shape, B, 1, k, 400 * 8)
+    csa.csa2_index_topk_reindex(shape, cache, B, qp, iq, pool, pool_n, k, out2, ws=ws2)
+    assert csa.csa2_get_device_status(ws2) == 0
+    for b in range(B):
+        oc = oracle_seq(seed, b, n, n, swa_cap)
+        qb = query_values(seed, "iq", [b], [qpos[b]], 256, "cpu")[0]
+        ridx, rpool, rpn = oc.index_topk_full(qpos[b], qb, k=k, pool_blocks=P, ratio=2)
+        assert int(opn[b]) == rpn
+        assert np.array_equal(opool[b].cpu().numpy(), rpool)
+        assert np.array_equal(out[b].cpu().numpy(), ridx)
+        rr = oc.index_topk_reindex(qpos[b], qb, pool[b].cpu().numpy(), int(pool_n[b]), k=k, ratio=2)
+        assert np.array_equal(out2[b].cpu().numpy(), rr)
