@@ -7,6 +7,19 @@ dequantisation and attention all run in the CUDA kernels of libcsa2.so. There is
 fallback: if the library is not built, loading fails loudly.
 
 Plumbing helpers (`Cache`, `Workspace`) allocate device memory with torch and fill the C structs.
+
+A Reindex decode step for a batch of B sequences (tensors on the GPU, bf16 unless noted):
+
+    shape = make_shape()                                  # 16 x 128 heads, indexer 4 x 64, window 128
+    cache = Cache(B, cap, swa_cap)                        # FP4 main / indexer planes + FP8 window ring
+    ws = Workspace(shape, B, 1, 512, pool_stride * 8)     # sized for the largest pool
+    csa2_quantize_append(shape, cache, B, t, pos, kv, idx_k, swa_kv)     # new entries (any plane may be None)
+    csa2_decode_reindex(shape, cache, B, qpos, swa_kv, idx_q, q, pool, pool_n, 512, idx, out, ws=ws)
+    status = csa2_get_device_status(ws)                   # bad indices / positions / pool ids, if any
+
+`out` [B, 16, 128] holds the attention output, `idx` [B, 512] the selected positions (ascending,
+-1 padded). The Full and Minimal modes, the separate index / attention calls and the prefill chunk
+follow the same pattern (include/csa2.h documents every argument).
 """
 from __future__ import annotations
 
