@@ -6,7 +6,7 @@
 // Fourfold", "Technical Approach": only Full mode writes main KV and indexer keys; every mode
 // writes its own sliding-window KV.
 //
-// Rounding (this build's reading of the unstated rule): s = E4M3_RNE_satfinite(amax / 6) in fp32,
+// Rounding (the reading taken here of a rule the pages leave open): s = E4M3_RNE_satfinite(amax / 6) in fp32,
 // all-zero codes when s == 0, code = E2M1_RNE_satfinite(x / s) with the sign of x kept.
 // The quotients are IEEE fp32 divisions; because x has 8 significant bits and s has 4, an fp32
 // quotient can never fall between a rounding boundary and the exact quotient, so these

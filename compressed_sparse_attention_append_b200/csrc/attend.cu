@@ -6,7 +6,7 @@
 //   sec. XI: cached values are dequantised before attention (E2M1 x E4M3 products are exact in
 //   fp16, and FP8 window values are exact in fp16, so the dequantised keys and values are exact);
 //   sec. XII: a query at position i sees window keys [max(s, i - win + 1), i].
-// This build's reading: one softmax over selected and window keys together, 16 query heads
+// Reading taken here: one softmax over selected and window keys together, 16 query heads
 // sharing one K/V head, default scale 1/sqrt(128).
 //
 // Per CTA: one query row and one split of its key list (valid selected entries in index order,

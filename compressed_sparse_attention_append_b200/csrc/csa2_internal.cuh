@@ -17,7 +17,7 @@
 
 namespace csa2 {
 
-// ---- fixed shapes of this build ---------------------------------------------------------------
+// ---- fixed shapes of this library -------------------------------------------------------------
 constexpr int kHQ = 16;       // query heads
 constexpr int kD = 128;       // head dim (K and V)
 constexpr int kKVBytes = 128; // packed E2M1 bytes of one main K||V row (256 channels)

@@ -6,7 +6,7 @@
 // Top-K indices. [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token",
 // sec. IX (the indexer scores every visible position), sec. XI: indexer queries and keys are FP4.
 //
-// Score (this build's reading; the pages give no formula): score(p) = sum_h q_h . k_{p,h} over 4
+// Score (the reading taken here; the pages give no formula): score(p) = sum_h q_h . k_{p,h} over 4
 // heads x 64 channels of dequantised FP4 values, computed EXACTLY as the integer S = score * 2^20:
 //   * an E2M1 code c decodes to the integer 2*value(c) in {0, +-1, +-2, +-3, +-4, +-6, +-8, +-12}
 //     through a byte permute (prmt) of the table {0,1,2,3,4,6,8,12}: the permute's sign-replicate

@@ -24,7 +24,7 @@
  *     capacity, a pool block id out of range) set bits of a status word inside the workspace
  *     and the offending item is skipped; read it with csa2_get_device_status. No call traps,
  *     asserts or spins on the device.
- *   - Fixed shapes of this build: hq = 16 query heads, d = 128 (K and V each), one shared KV
+ *   - Fixed shapes of this library: hq = 16 query heads, d = 128 (K and V each), one shared KV
  *     head, hi = 4 indexer query heads, di = 64, hk = 4 indexer key heads, bs = 8 positions
  *     per pool block, win <= 128. Other values return CSA2_ERR_UNSUPPORTED_SHAPE.
  */
@@ -47,7 +47,7 @@ extern "C" {
 typedef enum {
     CSA2_OK = 0,
     CSA2_ERR_INVALID_ARG = 1,      /* null pointer, negative size, misaligned pointer        */
-    CSA2_ERR_UNSUPPORTED_SHAPE = 2,/* shape outside what this build implements               */
+    CSA2_ERR_UNSUPPORTED_SHAPE = 2,/* shape outside what this library implements             */
     CSA2_ERR_CAPACITY = 3,         /* a bound that the host can see exceeds the cache        */
     CSA2_ERR_WORKSPACE = 4,        /* workspace pointer null or smaller than required        */
     CSA2_ERR_CUDA = 5,             /* a kernel launch failed (cudaGetLastError)              */
@@ -77,7 +77,7 @@ typedef struct {
 } csa2_shape;
 
 /*
- * Cache of `batch` sequences (layout fixed by this build; the pages give none). Per sequence b
+ * Cache of `batch` sequences (layout fixed by this library; the pages give none). Per sequence b
  * and position p (0 <= p < cap):
  *   kv_data  + (b*cap + p)*128      : main K||V, 256 channels (K = 0..127, V = 128..255) as E2M1
  *                                     codes, channel 2j in the low nibble of byte j
@@ -133,7 +133,7 @@ CSA2_API csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream
  *   kv     [batch][t][256] bf16 or NULL  -> kv_data / kv_scale
  *   idx_k  [batch][t][hk*64] bf16 or NULL -> ik_data / ik_scale
  *   swa_kv [batch][t][256] bf16 or NULL  -> swa ring slots (pos+i) & (swa_cap-1)
- * Rounding (this build's reading): per 16-channel block s = E4M3_RNE_satfinite(amax/6);
+ * Rounding (the reading taken here): per 16-channel block s = E4M3_RNE_satfinite(amax/6);
  * s == 0 gives all-zero codes; code_i = E2M1_RNE_satfinite(x_i / s) keeping the sign of x_i;
  * SWA bytes = E4M3_RNE_satfinite(x). A sequence whose range leaves [0, cap) sets
  * CSA2_DEV_BAD_POS and is skipped (needs `ws`; pass NULL to skip the device check).
@@ -156,7 +156,7 @@ CSA2_API csa2_status csa2_quantize_append(const csa2_shape* shape, const csa2_ca
  *   out_pool [batch][P] int32 : pool block ids, ascending, padded with -1 (NULL if P == 0)
  *   out_pool_n [batch] int32 : min(P, ceil(visible entries / bs))  (NULL if P == 0)
  *   max_ctx  : host upper bound on the visible entries over all rows (<= cap)
- * Score (this build's reading): score(p) = sum_h q_h . k_{p,h} on dequantised values, exact;
+ * Score (the reading taken here): score(p) = sum_h q_h . k_{p,h} on dequantised values, exact;
  * ranking by score descending, ties to the lower position (lower block id for the pool).
  */
 CSA2_API csa2_status csa2_index_topk_full(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
@@ -189,7 +189,7 @@ CSA2_API csa2_status csa2_index_topk_reindex(const csa2_shape* shape, const csa2
  *   sm_scale : softmax scale, 0 gives 1/sqrt(d)
  *   out [batch][tq][hq][d] bf16; out_f32 (same shape, fp32) and lse [batch][tq][hq] fp32 (natural
  *   log) may be NULL.
- * This build's reading: ONE softmax over selected rows and window rows together; a position may
+ * Reading taken here: ONE softmax over selected rows and window rows together; a position may
  * appear in both (its FP4 main entry and its FP8 window entry are different vectors). An index
  * < -1, not visible at qpos (see ratio) or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row with no key gives out = 0
  * and lse = -inf.

@@ -45,7 +45,7 @@
  * rational arithmetic, library routines (torch float8 conversion, Python sorted(), torch
  * fp64 softmax attention), closed forms and the byte figures printed in [C] sec. VII.
  * The R2/R3/R7 semantics (score formula, key heads, one softmax over selected + window)
- * are this build's definitions: no page figure can confirm them ("parity unpinned" as to
+ * are definitions stated here: no page figure can confirm them ("parity unpinned" as to
  * the pages; pinned as to the definitions stated here).
  */
 #include <math.h>

@@ -10,7 +10,7 @@ from conftest import golden
 
 
 def test_entry_bytes_rule(orc):
-    assert orc.entry_bytes(256) == 144  # main K||V row of this build: 128 B codes + 16 B scales
+    assert orc.entry_bytes(256) == 144  # main K||V row of this library: 128 B codes + 16 B scales
     assert orc.entry_bytes(64) == 36
     assert orc.entry_bytes(512) == 288
     assert orc.entry_bytes(0) == 0 and orc.entry_bytes(100) == 0
