@@ -120,7 +120,7 @@ class Clocks:
 
     def summary(self):
         if not self.proc or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
@@ -136,6 +136,156 @@ class Clocks:
         sm.sort()
         return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# NVML clock-event reason bits (nvmlClocksEventReason*), by the names the clock record uses
+NVML_REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+                ("sw_power_cap", 0x4))
+
+
+def nvml_clock_summary(samples, window, max_mhz):
+    """Median SM clock and the union of reasons over the (time, sm_mhz, reason_bits) samples that
+    fall inside window = (t0, t1); None when no sample does."""
+    t0, t1 = window
+    inside = [s for s in samples if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+    if not inside:
+        return None
+    sm = sorted(s[1] for s in inside)
+    bits = 0
+    for s in inside:
+        bits |= s[2]
+    return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max_mhz,
+            "reasons": sorted(n for n, b in NVML_REASONS if bits & b), "samples": len(inside)}
+
+
+def nvml_sample_loop(nv, handle, period, out, stop=lambda: False):
+    """Writes one line "time sm_mhz reason_bits" per NVML reading of the SM clock and the
+    clock-event reasons to the open file `out`, every `period` seconds, until stop() is true.
+    Time is time.monotonic(), the same clock in every process of the host. Reads only."""
+    reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+        nv.nvmlDeviceGetCurrentClocksThrottleReasons
+    while not stop():
+        t = time.monotonic()
+        sm = int(nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM))
+        bits = int(reasons(handle))
+        out.write(f"{t:.6f} {sm} {bits}\n")
+        out.flush()
+        time.sleep(period)
+
+
+def nvml_sampler_main(uuid, bus, period, path):
+    """Body of the sampler process: the NVML device with this UUID (else this PCI address); the
+    file gets "max <MHz>" first, then nvml_sample_loop's lines until the process is ended."""
+    import pynvml
+
+    pynvml.nvmlInit()
+    try:
+        h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+    except Exception:
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+    with open(path, "w") as f:
+        f.write(f"max {int(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))}\n")
+        f.flush()
+        nvml_sample_loop(pynvml, h, period, f)
+
+
+def read_nvml_samples(path):
+    """(samples [(time, sm_mhz, reason_bits)], max_mhz) from a sampler file; complete lines only."""
+    samples, mx = [], None
+    try:
+        with open(path) as f:
+            for line in f:
+                c = line.split()
+                if not line.endswith("\n"):
+                    break
+                if len(c) == 2 and c[0] == "max":
+                    mx = int(c[1])
+                elif len(c) == 3:
+                    samples.append((float(c[0]), int(c[1]), int(c[2])))
+    except OSError:
+        pass
+    return samples, mx
+
+
+class NvmlClocks:
+    """SM clock and clock-event reasons of one GPU, read through NVML about every `period` seconds
+    by a separate process (so that sampling takes nothing from the process that launches the
+    kernels); summary() keeps the samples taken between mark_start() and mark_end(). The timed
+    region of a decode step lasts milliseconds, far below nvidia-smi's sampling period, so this is
+    the record that can see inside it. Reads only: no clock or setting is changed."""
+
+    def __init__(self, ident=None, period=0.001, path=None, start_timeout=10.0):
+        self.ident, self.period, self.start_timeout = ident, period, start_timeout
+        d = os.environ.get("CSA2_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = path or os.path.join(d, f"csa2_nvml_{os.getpid()}.txt")
+        self.proc = None
+        self.window = [None, None]
+
+    @classmethod
+    def for_device(cls, device, **kw):
+        """Sampler of the NVML device that is CUDA device `device` (matched by UUID, else by PCI
+        address); one that records nothing when the device properties are unavailable."""
+        try:
+            import torch
+
+            p = torch.cuda.get_device_properties(device)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            return cls(("GPU-" + str(p.uuid), bus), **kw)
+        except Exception:
+            return cls(None, **kw)
+
+    def __enter__(self):
+        if self.ident is None:
+            return self
+        try:
+            if os.path.exists(self.path):
+                os.remove(self.path)
+            code = (f"import sys; sys.path.insert(0, {ROOT!r}); import bench; "
+                    f"bench.nvml_sampler_main({self.ident[0]!r}, {self.ident[1]!r}, {self.period!r}, {self.path!r})")
+            self.proc = subprocess.Popen([sys.executable, "-c", code], stdout=subprocess.DEVNULL,
+                                         stderr=subprocess.DEVNULL)
+            t0 = time.monotonic()
+            while time.monotonic() - t0 < self.start_timeout and self.proc.poll() is None:
+                if len(read_nvml_samples(self.path)[0]) >= 2:
+                    break
+                time.sleep(0.02)
+        except Exception:
+            self.proc = None
+        return self
+
+    def mark_start(self):
+        self.window[0] = time.monotonic()
+
+    def mark_end(self):
+        self.window[1] = time.monotonic()
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        self._summary = self.summary()
+        if not os.environ.get("CSA2_CLOCKS_DIR") and os.path.exists(self.path):
+            os.remove(self.path)  # kept only where the samples were asked for
+
+    def summary(self):
+        if getattr(self, "_summary", None) is not None:
+            return self._summary
+        samples, mx = read_nvml_samples(self.path)
+        return nvml_clock_summary(samples, tuple(self.window), mx)
+
+
+def clocks_record(nvml, smi):
+    """The clocks object of the JSON line: NVML samples inside the timed region when there are any,
+    else nvidia-smi's samples around it; both sources' sample counts are given."""
+    s = smi.summary()
+    n = nvml.summary()
+    if n is None:
+        return dict(s, source="nvidia-smi -lms 100 around the timed region")
+    return dict(n, source="NVML every ~1 ms from the launch of the timed region to its end", smi_samples=s.get("samples", 0),
+                smi_sm_mhz=s.get("sm_mhz"), smi_reasons=s.get("reasons"))
 
 
 # ---------------------------------------------------------------------------------------------
@@ -225,7 +375,7 @@ def run_gpu(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=600))
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     wl = W.WORKLOADS[args.workload]
     B = args.batch or wl.batch
@@ -239,12 +389,6 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    # warm-up
-    for _ in range(args.warmup):
-        step.run()
-    barrier()
-
-    # ---- timed region: K steps, per-kernel events on the launching stream ----
     kern = ("append", "index", "attend") if wl.mode != "prefill" else ("prefill",)
     ev = {k: [] for k in kern}
 
@@ -257,9 +401,14 @@ def run_gpu(args):
             ev[name][-1][1] = e
 
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with Clocks(local) as clk:
+    # the clock samplers start before the warm-up, so that they are running when the timed region is
+    with Clocks(local) as clk, NvmlClocks.for_device(dev) as nclk:
+        for _ in range(args.warmup):
+            step.run()
         barrier()
+        # ---- timed region: K steps, per-kernel events on the launching stream ----
         torch.cuda._sleep(int(2e7))  # lets the host enqueue the K steps ahead of the GPU
+        nclk.mark_start()
         start.record(stream)
         for _ in range(args.steps):
             if wl.mode == "prefill":
@@ -270,6 +419,7 @@ def run_gpu(args):
                 step.run_parts(hook)
         end.record(stream)
         barrier()
+        nclk.mark_end()
     ms = start.elapsed_time(end)
     kms = {k: sum(a.elapsed_time(b) for a, b in v) / max(1, len(v)) for k, v in ev.items()}
     ms_max = reduce_max(ms, dev, world)
@@ -336,7 +486,7 @@ def run_gpu(args):
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": launches,
-        "clocks": clk.summary(),
+        "clocks": clocks_record(nclk, clk),
     }
     if world == 1 and not args.no_cpu_baseline:
         v, desc, cores = oracle_sample(args.workload, budget_s=args.cpu_budget, context=args.context or None)
