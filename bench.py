@@ -198,10 +198,13 @@ def read_nvml_samples(path):
                 c = line.split()
                 if not line.endswith("\n"):
                     break
-                if len(c) == 2 and c[0] == "max":
-                    mx = int(c[1])
-                elif len(c) == 3:
-                    samples.append((float(c[0]), int(c[1]), int(c[2])))
+                try:
+                    if len(c) == 2 and c[0] == "max":
+                        mx = int(c[1])
+                    elif len(c) == 3:
+                        samples.append((float(c[0]), int(c[1]), int(c[2])))
+                except ValueError:
+                    continue
     except OSError:
         pass
     return samples, mx
@@ -267,8 +270,11 @@ class NvmlClocks:
             except Exception:
                 self.proc.kill()
         self._summary = self.summary()
-        if not os.environ.get("CSA2_CLOCKS_DIR") and os.path.exists(self.path):
-            os.remove(self.path)  # kept only where the samples were asked for
+        if not os.environ.get("CSA2_CLOCKS_DIR"):
+            try:
+                os.remove(self.path)  # kept only where the samples were asked for
+            except OSError:
+                pass
 
     def summary(self):
         if getattr(self, "_summary", None) is not None:
