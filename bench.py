@@ -47,6 +47,10 @@ def algorithmic_bytes(wl):
     elif wl.mode == "minimal":
         index = 0
         append = 256 * 2 + 256
+    elif wl.mode == "draft":
+        # the tq rows of a sequence share one pass over its visible indexer keys: per row, 1/tq of it
+        index = wl.context * 144 / wl.tq + iq + idx
+        append = 3 * 256 * 2 + 144 * 2 + 256
     else:
         index = wl.context * 144 + iq + idx  # per query row (upper bound: the last row sees all)
         append = 3 * 256 * 2 + 144 * 2 + 256
@@ -308,16 +312,19 @@ def oracle_sample(wl_name, budget_s=12.0, context=None, seqs=(0, 1)):
     seqs = list(seqs)
     built = [OW.build_sequence(wl, b) for b in seqs]
     rows = [0] if wl.mode == "prefill" else None
+    per_step = 1 if wl.mode == "prefill" else wl.tq  # queries one oracle step answers
     n = 0
     t0 = time.perf_counter()
     while True:
         for c, inp in built:
             OW.run_step(c, wl, inp, rows=rows)
-            n += 1
+            n += per_step
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    what = "prefill query rows (one row per step)" if wl.mode == "prefill" else "whole decode steps"
+    what = {"prefill": "prefill query rows (one row per step)",
+            "draft": f"query rows of whole multi-token decode steps ({wl.tq} rows per step)"}.get(wl.mode,
+                                                                                             "whole decode steps")
     desc = (f"{n} {what} of {wl_name} (sequences {seqs} repeated, cache resident in host memory), "
             f"single-threaded C oracle, fp64, {el:.1f} s")
     return n / el, desc, 1
@@ -430,7 +437,8 @@ def run_gpu(args):
     kms = {k: sum(a.elapsed_time(b) for a, b in v) / max(1, len(v)) for k, v in ev.items()}
     ms_max = reduce_max(ms, dev, world)
     value = weak_value(B * wl.tq, world, args.steps, ms_max)
-    # kernels per step: append 1; index (decode rows) zero + score + select = 3, (prefill) 1; attend 1
+    # kernels per step: append 1; index (decode rows) zero + score + select = 3, (several rows per
+    # sequence: prefill, draft) 1; attend 1
     per_step = {"full": 5, "reindex": 5, "minimal": 2}.get(wl.mode, 3)
     launches = args.steps * per_step
     if wl.mode == "minimal":
@@ -447,10 +455,13 @@ def run_gpu(args):
 
     peak, peak_kind = measured_peaks()
     ab = algorithmic_bytes(wl)
-    dom = "index" if wl.mode in ("full", "reindex") else ("attend" if wl.mode == "minimal" else "prefill")
+    dom = "index" if wl.mode in ("full", "reindex", "draft") else ("attend" if wl.mode == "minimal" else "prefill")
     if dom == "prefill":
         dom_bytes = (ab["index"] + ab["attend"]) * wl.tq
         dom_file, dom_kernels = "index.cu", "index_kernel + attend_kernel"
+    elif wl.mode == "draft":
+        dom_bytes = int(round(ab[dom] * B * wl.tq))
+        dom_file, dom_kernels = "index.cu", "index_kernel"
     else:
         dom_bytes = ab[dom] * B
         # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
@@ -481,7 +492,8 @@ def run_gpu(args):
         "warmup": args.warmup, "ms_per_step": round(ms_max / args.steps, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic (seeded near-Gaussian bf16, sigma 1, clipped to +-26)",
-        "config": {"workload": args.workload + (f"@ctx{wl.context}" if args.context else ""), "mode": wl.mode, "batch_per_gpu": B, "context": wl.context,
+        "config": {"workload": args.workload + (f"@ctx{wl.context}" if args.context else ""), "mode": wl.mode,
+                   "batch_per_gpu": B, "query_rows_per_sequence": wl.tq, "context": wl.context,
                    "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": 16, "head_dim": 128,
                    "indexer": "4 heads x 64, FP4", "kv_cache": "E2M1 + E4M3/16 (FP4), window FP8",
                    "window": wl.win, "parallelism": f"dp{world}",
@@ -510,7 +522,7 @@ def run_e2e(step, args, world, barrier):
     if wl.mode == "prefill":
         names_in = ["kv", "idx_k", "swa_kv", "idx_q", "q"]
     else:
-        names_in = [n for n in ("qpos", "swa_kv", "idx_q", "q", "pool", "pool_n", "kv", "idx_k", "idx")
+        names_in = [n for n in ("pos", "qpos", "swa_kv", "idx_q", "q", "pool", "pool_n", "kv", "idx_k", "idx")
                     if n in step.inputs]
     host_in = {n: step.inputs[n].cpu().pin_memory() for n in names_in}
     names_out = ["out"] + (["idx"] if "idx" in step.outputs and wl.mode != "minimal" else [])
@@ -540,7 +552,16 @@ def run_e2e(step, args, world, barrier):
     ms = reduce_max(s.elapsed_time(e), "cuda", world)
     v = weak_value(step.batch * wl.tq, world, K, ms)
     return {"value": round(v, 1), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": round(ms / K, 5), "call": f"csa2_decode_{wl.mode}" if wl.mode != "prefill" else "csa2_prefill_chunk"}
+            "ms_per_step": round(ms / K, 5), "call": e2e_call(wl.mode)}
+
+
+def e2e_call(mode):
+    """The public entry point(s) one end-to-end step goes through."""
+    if mode == "prefill":
+        return "csa2_prefill_chunk"
+    if mode == "draft":
+        return "csa2_quantize_append + csa2_index_topk_full + csa2_sparse_attend (tq rows)"
+    return f"csa2_decode_{mode}"
 
 
 def run_reference(args):

@@ -1,4 +1,4 @@
-"""The oracle's side of the five workloads: one sequence's cache and one step, regenerated on the host
+"""The oracle's side of the workloads: one sequence's cache and one step, regenerated on the host
 from the seeded generator (workloads/__init__.py), positions filled exactly as the GPU builder fills
 them. TEST INFRASTRUCTURE (tests, smoke and bench.py's CPU baseline only)."""
 from __future__ import annotations
@@ -29,6 +29,19 @@ def build_sequence(wl, b):
     if wl.mode == "prefill":
         p0 = N - wl.tq
         c = SeqCache(cap=N, swa_cap=1 << (wl.tq + wl.win - 1).bit_length())
+        for a in range(0, p0, 16384):
+            p = torch.arange(a, min(p0, a + 16384))
+            c.append(a, kv=_v(seed, "kv", b, p, 256), idx_k=_v(seed, "ik", b, p, 256))
+        pw = torch.arange(p0 - wl.win, p0)
+        c.append(p0 - wl.win, swa_kv=_v(seed, "swa", b, pw, 256))
+        p = torch.arange(p0, N)
+        for n, s, w in (("kv", "kv", 256), ("idx_k", "ik", 256), ("swa_kv", "swa", 256), ("idx_q", "iq", 256),
+                        ("q", "q", 2048)):
+            inp[n] = _v(seed, s, b, p, w)
+        return c, inp
+    if wl.mode == "draft":
+        p0 = N - wl.tq
+        c = SeqCache(cap=N, swa_cap=1 << (wl.tq + wl.win - 1).bit_length(), hk=4)
         for a in range(0, p0, 16384):
             p = torch.arange(a, min(p0, a + 16384))
             c.append(a, kv=_v(seed, "kv", b, p, 256), idx_k=_v(seed, "ik", b, p, 256))
@@ -71,14 +84,16 @@ def build_sequence(wl, b):
 
 
 def run_step(c, wl, inp, rows=None):
-    """One decode step (or the listed prefill rows) of the oracle. Returns a dict of results."""
+    """One decode step (or the listed rows of a prefill chunk or a multi-token decode; all rows when
+    rows is None) of the oracle. Returns a dict of results: idx/out/lse for one-row decode, else
+    rows = {row: (idx, out, lse)}."""
     N = wl.context
     r = {}
-    if wl.mode == "prefill":
+    if wl.mode in ("prefill", "draft"):
         p0 = N - wl.tq
         c.append(p0, kv=inp["kv"], idx_k=inp["idx_k"], swa_kv=inp["swa_kv"])
         r["rows"] = {}
-        for i in rows:
+        for i in (range(wl.tq) if rows is None else rows):
             idx = c.index_topk_full(p0 + i, inp["idx_q"][i], k=wl.k)
             r["rows"][i] = (idx,) + c.sparse_attend(p0 + i, inp["q"][i], idx)
         return r

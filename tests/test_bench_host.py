@@ -147,3 +147,14 @@ def test_reindex_algorithmic_bytes_per_query():
 @pytest.mark.parametrize("v,expect", [(1.0, 1), (-3.5, -3.5)])
 def test_reduce_max_single_rank_is_identity(v, expect):
     assert bench.reduce_max(v, "cpu", 1) == expect
+
+
+def test_draft_rows_share_one_pass_over_the_keys():
+    import workloads as W
+
+    wl = W.WORKLOADS["draft_b64_n131072_tq5"]
+    ab = bench.algorithmic_bytes(wl)
+    # per step and sequence: every visible indexer row once, plus each row's query and indices
+    assert ab["index"] * wl.tq == 131072 * 144 + 5 * (4 * 64 * 2 + 512 * 4)
+    assert bench.e2e_call("draft").startswith("csa2_quantize_append")
+    assert bench.e2e_call("reindex") == "csa2_decode_reindex"

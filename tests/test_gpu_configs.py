@@ -1,6 +1,6 @@
-"""The five workloads at full size, in the launch configuration bench.py times, checked on sampled
-sequences (prefill: sampled query rows) against the oracle: index sets and pools identical, attention
-within tolerance."""
+"""The workloads at full size, in the launch configuration bench.py times, checked on sampled
+sequences (prefill: sampled query rows; multi-token decode: every row of sampled sequences) against
+the oracle: index sets and pools identical, attention within tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -65,5 +65,30 @@ def test_prefill_workload_sampled_rows(orc):
         idx, ro, _ = r["rows"][i]
         assert np.array_equal(step.outputs["idx"][i].cpu().numpy(), idx), i
         _cmp_attn(step.outputs["out"][i], of[i], ro)
+    del step
+    torch.cuda.empty_cache()
+
+
+def test_draft_workload_sampled(orc):
+    """Multi-token decode (5 draft tokens per sequence, 64 sequences at N = 131,072): the three calls
+    bench.py times; every row of sampled sequences against the oracle."""
+    import compressed_sparse_attention_append_b200 as csa
+
+    step = G.build("draft_b64_n131072_tq5")
+    wl = step.wl
+    of = torch.empty(step.batch, wl.tq, 16, 128, dtype=torch.float32, device="cuda")
+    step.run(out_f32=of)
+    assert csa.csa2_get_device_status(step.ws) == 0
+    for b in (0, 63):
+        c, inp = OW.build_sequence(wl, b)
+        r = OW.run_step(c, wl, inp)
+        for t in range(wl.tq):
+            idx, ro, _ = r["rows"][t]
+            assert np.array_equal(step.outputs["idx"][b, t].cpu().numpy(), idx), (b, t)
+            _cmp_attn(step.outputs["out"][b, t], of[b, t], ro)
+    prev = {k: v.clone() for k, v in step.outputs.items()}
+    step.run()
+    for k, v in step.outputs.items():
+        assert torch.equal(v, prev[k]), k
     del step
     torch.cuda.empty_cache()

@@ -61,3 +61,28 @@ def test_distinct_sorted_sets():
 def test_cache_counters_layout():
     c = W.cache_counters(torch.tensor([0, 2]), torch.tensor([[5], [7]]), 4)
     assert c.tolist() == [[[20, 21, 22, 23]], [[((2 << 21) + 7) * 4 + i for i in range(4)]]]
+
+
+def test_draft_rows_are_causal_in_the_oracle_driver(orc):
+    """Multi-token decode on the oracle side, at a small context: row t of a step that appended all 5
+    draft tokens equals row t of a step whose cache holds only the tokens up to N-5+t, and every
+    selected position of row t is visible to it."""
+    from oracle import workload as OW
+
+    wl = OW.workload("draft_b64_n131072_tq5", context=2048)
+    p0 = wl.context - wl.tq
+    c, inp = OW.build_sequence(wl, 3)
+    r = OW.run_step(c, wl, inp)
+    assert sorted(r["rows"]) == list(range(wl.tq))
+    for t in range(wl.tq):
+        idx, out, lse = r["rows"][t]
+        sel = idx[idx >= 0]
+        assert sel.size == wl.k and sel.max() <= p0 + t and np.all(np.diff(sel) > 0)
+        c2, inp2 = OW.build_sequence(wl, 3)
+        c2.append(p0, kv=inp2["kv"][:t + 1], idx_k=inp2["idx_k"][:t + 1], swa_kv=inp2["swa_kv"][:t + 1])
+        idx2 = c2.index_topk_full(p0 + t, inp2["idx_q"][t], k=wl.k)
+        out2, lse2 = c2.sparse_attend(p0 + t, inp2["q"][t], idx2)
+        assert np.array_equal(idx, idx2)
+        assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
+    # the rows differ: each sees one more token and has its own query
+    assert not np.array_equal(r["rows"][0][1], r["rows"][wl.tq - 1][1])

@@ -5,7 +5,7 @@ This module holds none of the method's arithmetic. It only produces:
     uniforms, i.e. Irwin-Hall(12), unit variance, support +-6 sigma), scaled by sigma and
     clipped to +-clip (the pages bound post-RoPE magnitudes by about 26);
   * random distinct position / block-id sets, emitted in ascending order;
-  * the shapes of the five workloads.
+  * the shapes of the workloads (five layer-step configurations and a multi-token decode).
 
 Every value is a pure function of (seed, stream, counter) built from integer operations,
 one exact power-of-two scaling, one fp32 multiply by sigma, a clamp and one fp32 -> bf16
@@ -113,13 +113,13 @@ def distinct_sorted(seed: int, stream, b: torch.Tensor, n_range: int, count: int
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str            # "full" | "reindex" | "minimal" | "prefill"
+    mode: str            # "full" | "reindex" | "minimal" | "prefill" | "draft"
     batch: int
     context: int         # N: visible positions for a decode query (query at N-1)
     seed: int
     k: int = 512
     pool_blocks: int = 0  # Full: blocks kept in the pool; Reindex: blocks given
-    tq: int = 1           # query rows per sequence (prefill chunk length)
+    tq: int = 1           # query rows per sequence (prefill chunk length, draft tokens verified)
     hq: int = 16
     d: int = 128
     hi: int = 4
@@ -136,4 +136,7 @@ WORKLOADS = {
     "reindex_b128_n1m": Workload("reindex_b128_n1m", "reindex", 128, 1 << 20, seed=2, pool_blocks=2000),
     "minimal_b256_n262144": Workload("minimal_b256_n262144", "minimal", 256, 262144, seed=3),
     "prefill_t4096_at_1m": Workload("prefill_t4096_at_1m", "prefill", 1, (1 << 20) + 4096, seed=4, tq=4096),
+    # multi-token decode: each sequence appends 5 draft tokens at N-5 .. N-1 and verifies them together
+    # (Full index over every visible position, row t sees positions <= N-5+t; no block pool)
+    "draft_b64_n131072_tq5": Workload("draft_b64_n131072_tq5", "draft", 64, 131072, seed=5, tq=5),
 }

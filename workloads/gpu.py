@@ -1,4 +1,4 @@
-"""Builds the five workloads on a GPU through libcsa2's C ABI (bench.py and the full-size parity
+"""Builds the workloads on a GPU through libcsa2's C ABI (bench.py and the full-size parity
 tests use it). Inputs come from the seeded generator in workloads/__init__.py, made on the device;
 the cache is filled with libcsa2's own quantise-append. Only the positions a step can read are
 filled (a Reindex step reads only its pool, a Minimal step only its inherited rows); the rest of
@@ -45,10 +45,29 @@ class Step:
         elif wl.mode == "minimal":
             csa.csa2_decode_minimal(self.shape, self.cache, self.batch, I["qpos"], I["swa_kv"], I["q"], I["idx"],
                                     wl.k, O["out"], out_f32=out_f32, lse=lse, ws=ws, stream=stream)
+        elif wl.mode == "draft":
+            self._draft(lambda n, ph: None, stream, ws, out_f32, lse)
         else:
             csa.csa2_prefill_chunk(self.shape, self.cache, wl.context - wl.tq, wl.tq, I["kv"], I["idx_k"],
                                    I["swa_kv"], I["idx_q"], I["q"], wl.k, O["idx"], O["out"], out_f32=out_f32,
                                    lse=lse, ws=ws, stream=stream)
+
+    def _draft(self, hooks, stream, ws, out_f32=None, lse=None):
+        """Multi-token decode: append the tq draft tokens, index tq rows, attend tq rows (there is no
+        composed entry point for tq > 1: these are the three calls a user makes)."""
+        wl, I, O, b, t = self.wl, self.inputs, self.outputs, self.batch, self.wl.tq
+        hooks("append", 0)
+        csa.csa2_quantize_append(self.shape, self.cache, b, t, I["pos"], I["kv"], I["idx_k"], I["swa_kv"], ws=ws,
+                                 stream=stream)
+        hooks("append", 1)
+        hooks("index", 0)
+        csa.csa2_index_topk_full(self.shape, self.cache, b, t, I["qpos"], I["idx_q"], wl.k, O["idx"],
+                                 max_ctx=self.max_ctx, ws=ws, stream=stream)
+        hooks("index", 1)
+        hooks("attend", 0)
+        csa.csa2_sparse_attend(self.shape, self.cache, b, t, I["qpos"], I["q"], O["idx"], wl.k, O["out"],
+                               out_f32=out_f32, lse=lse, ws=ws, stream=stream)
+        hooks("attend", 1)
 
     # ---- the same pass as separate entry points (kernel-level timing) ----
     def run_parts(self, hooks, stream=None):
@@ -57,6 +76,8 @@ class Step:
         b = self.batch
         if wl.mode == "prefill":
             raise NotImplementedError("prefill is timed through csa2_prefill_chunk")
+        if wl.mode == "draft":
+            return self._draft(hooks, stream, self.ws)
         hooks("append", 0)
         if wl.mode == "full":
             csa.csa2_quantize_append(self.shape, self.cache, b, 1, I["qpos"], I["kv"], I["idx_k"], I["swa_kv"],
@@ -109,6 +130,25 @@ def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda
         O["out"] = torch.empty(wl.tq, 16, 128, dtype=torch.bfloat16, device=device)
         ws = csa.Workspace(shape, 1, wl.tq, wl.k, N)
         return Step(wl, shape, cache, ws, I, O, 1, N)
+
+    if wl.mode == "draft":
+        T = wl.tq
+        p0 = N - T
+        cache = csa.Cache(B, N, 1 << (T + wl.win - 1).bit_length(), device=device)
+        _fill_range(cache, shape, wl.seed, seqs, 0, p0, device)
+        p = torch.arange(p0, N, device=device)
+        I["pos"] = torch.full((B,), p0, dtype=torch.int64, device=device)
+        I["qpos"] = p.unsqueeze(0).repeat(B, 1).contiguous()
+        I["kv"] = _vals(wl.seed, "kv", seqs, p, 256).contiguous()
+        I["idx_k"] = _vals(wl.seed, "ik", seqs, p, 256).contiguous()
+        I["swa_kv"] = _vals(wl.seed, "swa", seqs, p, 256).contiguous()
+        I["idx_q"] = _vals(wl.seed, "iq", seqs, p, 256).contiguous()
+        I["q"] = _vals(wl.seed, "q", seqs, p, 2048).reshape(B, T, 16, 128).contiguous()
+        O["idx"] = torch.empty(B, T, wl.k, dtype=torch.int32, device=device)
+        O["out"] = torch.empty(B, T, 16, 128, dtype=torch.bfloat16, device=device)
+        ws = csa.Workspace(shape, B, T, wl.k, N)
+        torch.cuda.synchronize()
+        return Step(wl, shape, cache, ws, I, O, B, N)
 
     qpos = torch.full((B,), N - 1, dtype=torch.int64, device=device)
     I["qpos"] = qpos
