@@ -53,9 +53,12 @@ class _SeqCache(ctypes.Structure):
 
 
 def lib():
+    """The loaded oracle library: oracle/libcsa2_oracle.so, or the build of csa2_oracle.c that the
+    environment variable CSA2_ORACLE_LIB names (the planted-mistake tests load copies of the source
+    with one mistake planted in each)."""
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
+        L = ctypes.CDLL(os.environ.get("CSA2_ORACLE_LIB") or build())
         d, i, i64, vp = ctypes.c_double, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p
         sig = {
             "orc_e2m1_decode": (d, [i]),
