@@ -129,7 +129,7 @@ class Workload:
     bs: int = 8
 
 
-# The five workloads, shapes as stated for this hot path.
+# The five layer-step workloads, shapes as stated for this hot path, and a multi-token decode.
 WORKLOADS = {
     "full_b1_n4096": Workload("full_b1_n4096", "full", 1, 4096, seed=0),
     "full_b64_n131072": Workload("full_b64_n131072", "full", 64, 131072, seed=1, pool_blocks=2048),
