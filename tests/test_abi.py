@@ -43,6 +43,46 @@ def test_header_compiles_as_c():
                                "-o", os.path.join(d, "t.o")])
 
 
+def test_plain_c_program_links_and_calls_the_host_entry_points(L):
+    """A C program built against include/csa2.h and linked to libcsa2.so (no Python, no torch) calls
+    the host-only entry points; every call returns before anything touches a GPU."""
+    import subprocess
+    import tempfile
+
+    prog = r"""
+#include <stdio.h>
+#include "csa2.h"
+int main(void) {
+    csa2_shape s = {16, 128, 4, 64, 4, 128, 8, 1};
+    size_t ws = 0;
+    int st = csa2_workspace_size(&s, 128, 1, 512, 16000, 0, &ws);
+    csa2_shape bad = s;
+    bad.hq = 64;
+    size_t ws2 = 0;
+    int st2 = csa2_workspace_size(&bad, 1, 1, 512, 16000, 0, &ws2);
+    bad = s;
+    bad.ratio = 3;
+    int st3 = csa2_workspace_size(&bad, 1, 1, 512, 16000, 0, &ws2);
+    printf("%zu %d %d %zu %d %d %d %s\n", csa2_entry_bytes(256), csa2_version(), st, ws, st2, st3,
+           st2 == CSA2_ERR_UNSUPPORTED_SHAPE && st3 == CSA2_ERR_UNSUPPORTED_SHAPE,
+           csa2_status_string(CSA2_ERR_WORKSPACE));
+    return 0;
+}
+"""
+    libdir = os.path.dirname(csa.lib()._name)
+    with tempfile.TemporaryDirectory() as d:
+        c, exe = os.path.join(d, "p.c"), os.path.join(d, "p")
+        with open(c, "w") as f:
+            f.write(prog)
+        subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), c, "-o",
+                               exe, "-L", libdir, "-l:libcsa2.so", f"-Wl,-rpath,{libdir}"])
+        out = subprocess.run([exe], capture_output=True, text=True, timeout=60, check=True).stdout.split(maxsplit=7)
+    assert out[0] == "144" and out[1] == str(csa.csa2_version()) and out[2] == "0"
+    assert int(out[3]) == csa.csa2_workspace_size(csa.make_shape(), 128, 1, 512, 16000, 0)
+    assert out[6] == "1"
+    assert out[7].strip() == csa.csa2_status_string(csa.CSA2_ERR_WORKSPACE)
+
+
 def test_host_functions(L):
     assert csa.csa2_entry_bytes(256) == 144
     assert csa.csa2_entry_bytes(512) == 288
