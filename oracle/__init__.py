@@ -78,6 +78,12 @@ def lib():
             "orc_index_topk_full": (i, [vp, i64, vp, i, i, i, vp, i, i, vp, vp, i]),
             "orc_index_topk_reindex": (i, [vp, i64, vp, i, vp, i, i, i, i, vp, i]),
             "orc_sparse_attend": (i, [vp, i64, vp, i, vp, i, i64, i, d, vp, vp, i]),
+            "orc_e8m0_decode": (d, [i]),
+            "orc_mx_entry_bytes": (i64, [i]),
+            "orc_mx_quantize_rows": (None, [vp, i64, i, vp, vp]),
+            "orc_mx_dequant_rows": (None, [vp, vp, i64, i, vp]),
+            "orc_mx_index_topk_full": (i, [vp, vp, i64, i64, vp, i, i, i, vp, vp, i]),
+            "orc_latent_attend": (i, [vp, vp, i64, vp, i64, i64, vp, i, vp, i, i64, i, d, vp, vp, i]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -257,4 +263,93 @@ class SeqCache:
                                      float(sm_scale), _p(out), _p(lse), int(ratio))
         if nk < 0:
             raise ValueError("index out of range")
+        return out, lse
+
+
+# ---- the pages' own shapes: MXFP4 indexer key, 512-channel latent ([C] sec. VII, config list) ----
+def e8m0_decode(byte: int) -> float:
+    """E8M0 shared scale: 2^(byte - 127); 0xFF is NaN."""
+    return lib().orc_e8m0_decode(int(byte))
+
+
+def mx_entry_bytes(ch: int) -> int:
+    """[C] sec. VII: bytes of an MXFP4 entry of ch channels = ch/2 + ch/32 (0 if ch % 32)."""
+    return lib().orc_mx_entry_bytes(int(ch))
+
+
+def mx_quantize_rows(x, ch: int):
+    """R13 MXFP4 codec over rows of `ch` channels -> (packed data [rows, ch/2], E8M0 [rows, ch/32])."""
+    xb = _bf16_bits(x).reshape(-1, ch)
+    rows = xb.shape[0]
+    data = np.zeros((rows, ch // 2), np.uint8)
+    scale = np.zeros((rows, ch // 32), np.uint8)
+    lib().orc_mx_quantize_rows(_p(xb), rows, ch, _p(data), _p(scale))
+    return data, scale
+
+
+def mx_dequant_rows(data: np.ndarray, scale: np.ndarray, ch: int) -> np.ndarray:
+    data = np.ascontiguousarray(data, np.uint8).reshape(-1, ch // 2)
+    scale = np.ascontiguousarray(scale, np.uint8).reshape(-1, ch // 32)
+    out = np.zeros((data.shape[0], ch), np.float64)
+    lib().orc_mx_dequant_rows(_p(data), _p(scale), data.shape[0], ch, _p(out))
+    return out
+
+
+class LatentCache:
+    """One sequence's cache in the pages' own shapes: the 512-channel latent (K = V) in the R1 codec
+    (256 B of codes + 32 B of E4M3 scales per entry), the ONE 128-channel indexer key in MXFP4 (64 B
+    + 4 B of E8M0 scales per entry) and a power-of-two ring of 512-channel FP8 window rows."""
+
+    def __init__(self, cap: int, swa_cap: int):
+        assert swa_cap & (swa_cap - 1) == 0, "window ring capacity must be a power of two"
+        self.cap, self.swa_cap = cap, swa_cap
+        self.ldata = np.zeros((cap, 256), np.uint8)
+        self.lscale = np.zeros((cap, 32), np.uint8)
+        self.kdata = np.zeros((cap, 64), np.uint8)
+        self.kscale = np.zeros((cap, 4), np.uint8)
+        self.swa = np.zeros((swa_cap, 512), np.uint8)
+
+    def append(self, pos: int, latent=None, idx_k=None, swa=None):
+        """Quantise-append entries pos..pos+t-1 of any of the three planes (bf16 inputs)."""
+        if latent is not None:
+            xb = _bf16_bits(latent).reshape(-1, 512)
+            assert 0 <= pos and pos + xb.shape[0] <= self.cap
+            d, s = quantize_rows(xb, 512)
+            self.ldata[pos:pos + xb.shape[0]], self.lscale[pos:pos + xb.shape[0]] = d, s
+        if idx_k is not None:
+            xb = _bf16_bits(idx_k).reshape(-1, 128)
+            assert 0 <= pos and pos + xb.shape[0] <= self.cap
+            d, s = mx_quantize_rows(xb, 128)
+            self.kdata[pos:pos + xb.shape[0]], self.kscale[pos:pos + xb.shape[0]] = d, s
+        if swa is not None:
+            xb = _bf16_bits(swa).reshape(-1, 512)
+            for i in range(xb.shape[0]):
+                self.swa[(pos + i) & (self.swa_cap - 1)] = fp8_rows(xb[i])
+
+    def index_topk_full(self, qpos: int, idx_q, k: int = 512, relu=False, ratio: int = 1):
+        """R14: Top-k of the entries visible at token qpos for a 32 x 128 (any hi <= 64) query ->
+        (ascending positions padded with -1, scores of entries 0..visible-1)."""
+        qb = _bf16_bits(idx_q).reshape(-1, 128)
+        n = max(0, (qpos + 1) // ratio) if qpos >= 0 else 0
+        out = np.zeros(k, np.int32)
+        sc = np.zeros(max(n, 1), np.float64)
+        m = lib().orc_mx_index_topk_full(_p(self.kdata), _p(self.kscale), self.cap, int(qpos), _p(qb), qb.shape[0],
+                                         int(k), int(bool(relu)), _p(out), _p(sc), int(ratio))
+        assert m >= 0, "query outside the cache"
+        return out, sc[:n]
+
+    def attend(self, qpos: int, q, idx, swa_begin: int = 0, win: int = 128, sm_scale: float = 0.0, ratio: int = 1):
+        """R15: one softmax over the selected latent entries and the window rows, K = V = the latent;
+        sm_scale 0 means 1/sqrt(512). -> (out [hq, 512], lse [hq])."""
+        qb = _bf16_bits(q).reshape(-1, 512)
+        hq = qb.shape[0]
+        idx = np.ascontiguousarray(idx, np.int32)
+        if sm_scale == 0.0:
+            sm_scale = 1.0 / np.sqrt(512.0)
+        out = np.zeros((hq, 512), np.float64)
+        lse = np.zeros(hq, np.float64)
+        nk = lib().orc_latent_attend(_p(self.ldata), _p(self.lscale), self.cap, _p(self.swa), self.swa_cap, int(qpos),
+                                     _p(qb), hq, _p(idx), idx.size, int(swa_begin), int(win), float(sm_scale),
+                                     _p(out), _p(lse), int(ratio))
+        assert nk >= 0, "a selected entry is not visible or outside the cache"
         return out, lse

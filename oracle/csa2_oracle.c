@@ -40,6 +40,15 @@
  *   R12 compression ratio r in {1, 2}: cache entry e summarises tokens r*e .. r*e + r - 1 and is
  *       visible to a query at token i once all of them are <= i, i.e. the first floor((i + 1) / r)
  *       entries; the window stays per token.
+ *   R13 (the pages' own shapes) MXFP4 indexer key: per 32-channel block the shared E8M0 scale is
+ *       X = 2^(floor(log2 amax) - 2), the microscaling rule for E2M1 elements (whose largest value
+ *       is 1.5 * 2^2); elements E2M1_RNE_satfinite(x / X); amax == 0 gives scale byte 0 and +0 codes.
+ *   R14 (the pages' own shapes) indexer of 32 query heads x 128 channels over ONE shared 128-channel
+ *       key per entry (MQA); score = sum_h q_h . k (ReLU variant: sum_h max(0, q_h . k)); the query
+ *       goes through the same MXFP4 codec as the keys.
+ *   R15 (the pages' own shapes) attention over the 512-channel latent, which is both K and V, for
+ *       64 query heads of 512 channels; the latent in the R1 codec (288 B per entry), window rows
+ *       FP8 at 512 channels; one softmax over selected and window entries; scale 1/sqrt(512).
  *
  * Parity pins: every function here is checked by tests/test_oracle_*.py against exact
  * rational arithmetic, library routines (torch float8 conversion, Python sorted(), torch
@@ -420,5 +429,161 @@ ORC_API int orc_sparse_attend(const orc_seq_cache* c, int64_t qpos, const uint16
         lse[h] = (nk > 0) ? m + log(l) : -INFINITY;
     }
     free(K); free(V); free(lg);
+    return nk;
+}
+
+/* ==================================================================================== */
+/* The pages' own shapes ([C] sec. VII and the configuration list in its closing         */
+/* section): a 512-channel main KV latent that serves as both K and V for 64 query heads  */
+/* of dimension 512, and an indexer of 32 query heads of dimension 128 over ONE shared    */
+/* 128-channel key stored in MXFP4 (E2M1 elements, one E8M0 scale per 32 channels).       */
+/* ==================================================================================== */
+
+/* E8M0 (the microscaling shared scale): 2^(byte - 127); 0xFF is NaN. */
+ORC_API double orc_e8m0_decode(int byte)
+{
+    if ((byte & 0xFF) == 0xFF) return NAN;
+    return ldexp(1.0, (byte & 0xFF) - 127);
+}
+
+/* [C] sec. VII: bytes of an MXFP4 entry of `ch` channels = ch/2 (E2M1) + ch/32 (one E8M0 byte
+ * per 32 channels). Returns 0 when ch is not a multiple of 32. */
+ORC_API int64_t orc_mx_entry_bytes(int ch)
+{
+    if (ch <= 0 || ch % 32) return 0;
+    return ch / 2 + ch / 32;
+}
+
+/* MXFP4 quantiser (R13). Per 32-channel block: amax = max|x|; the shared scale is the power of
+ * two X = 2^(floor(log2 amax) - 2) (2 = the exponent of E2M1's largest value 6 = 1.5 * 2^2), its
+ * byte log2(X) + 127 clamped to 0..254; code_i = E2M1_RNE_satfinite(x_i / X) (x / X is exact).
+ * amax == 0 gives scale byte 0 and all codes +0. Packing as R9 (channel 2j low nibble). */
+ORC_API void orc_mx_quantize_rows(const uint16_t* x, int64_t rows, int ch, uint8_t* data, uint8_t* scale)
+{
+    int nb = ch / 32;
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t* xr = x + r * ch;
+        for (int b = 0; b < nb; ++b) {
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                double v = fabs(bf16_to_double(xr[32 * b + i]));
+                if (v > amax) amax = v;
+            }
+            int sbyte = 0;
+            if (amax > 0.0) {
+                int e2;
+                frexp(amax, &e2);                 /* amax in [2^(e2-1), 2^e2): floor(log2) = e2-1 */
+                sbyte = (e2 - 1) - 2 + 127;
+                if (sbyte < 0) sbyte = 0;
+                if (sbyte > 254) sbyte = 254;
+            }
+            scale[r * nb + b] = (uint8_t)sbyte;
+            double X = orc_e8m0_decode(sbyte);
+            for (int i = 0; i < 32; i += 2) {
+                int c0 = 0, c1 = 0;
+                if (amax > 0.0) {
+                    c0 = orc_e2m1_encode(bf16_to_double(xr[32 * b + i]) / X);
+                    c1 = orc_e2m1_encode(bf16_to_double(xr[32 * b + i + 1]) / X);
+                }
+                data[r * (ch / 2) + 16 * b + i / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+}
+
+/* Dequantise MXFP4 rows: v = E2M1(code) * E8M0(scale of the code's 32-channel block). */
+ORC_API void orc_mx_dequant_rows(const uint8_t* data, const uint8_t* scale, int64_t rows, int ch, double* out)
+{
+    int nb = ch / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int c = 0; c < ch; ++c) {
+            uint8_t byte = data[r * (ch / 2) + c / 2];
+            int code = (c & 1) ? (byte >> 4) : (byte & 15);
+            out[r * ch + c] = orc_e2m1_decode(code) * orc_e8m0_decode(scale[r * nb + c / 32]);
+        }
+}
+
+/* Indexer of the pages' shape (R14): the query (hi heads x 128 channels) goes through the same
+ * MXFP4 codec as the keys; score(p) = sum_h q_h . k_p over the ONE shared key of entry p (MQA);
+ * relu != 0 gives sum_h max(0, q_h . k_p). Keys: kdata [cap][64], kscale [cap][4]. Scores the
+ * entries visible at token qpos (R11, R12) and keeps the Top-k as orc_topk does (R5, R6). */
+ORC_API int orc_mx_index_topk_full(const uint8_t* kdata, const uint8_t* kscale, int64_t cap, int64_t qpos,
+                                   const uint16_t* idx_q, int hi, int k, int relu, int32_t* out_idx, double* out_scores,
+                                   int ratio)
+{
+    int64_t n = orc_visible(qpos, ratio);
+    if (n > cap || hi <= 0 || hi > 64) return -1;
+    uint8_t qdata[64 * 64], qscale[64 * 4];
+    double qd[64 * 128], kd[128];
+    orc_mx_quantize_rows(idx_q, hi, 128, qdata, qscale);
+    orc_mx_dequant_rows(qdata, qscale, hi, 128, qd);
+    int64_t* p = (int64_t*)malloc(sizeof(int64_t) * (n > 0 ? n : 1));
+    double* s = (double*)malloc(sizeof(double) * (n > 0 ? n : 1));
+    for (int64_t i = 0; i < n; ++i) {
+        p[i] = i;
+        orc_mx_dequant_rows(kdata + i * 64, kscale + i * 4, 1, 128, kd);
+        double total = 0.0;
+        for (int h = 0; h < hi; ++h) {
+            double dot = 0.0;
+            for (int c = 0; c < 128; ++c) dot += qd[h * 128 + c] * kd[c];
+            total += (relu && dot < 0.0) ? 0.0 : dot;
+        }
+        s[i] = total;
+        if (out_scores) out_scores[i] = total;
+    }
+    int m = orc_topk(s, p, n, k, out_idx);
+    free(p); free(s);
+    return m;
+}
+
+/* Attention of the pages' shape (R15): the 512-channel latent is both K and V. Main entries:
+ * ldata [cap][256] E2M1 codes + lscale [cap][32] E4M3 scales (the R1 codec at 512 channels,
+ * 288 B per entry); window entries: swa [swa_cap][512] E4M3 without scale, slot = pos &
+ * (swa_cap - 1). A query at token qpos with hq heads of 512 channels attends, in ONE softmax,
+ * to the selected entries (idx, -1 skipped; each must be visible, R12) and the window tokens
+ * [max(swa_begin, qpos - win + 1), qpos]; logits (q_h . l_j) * sm_scale; out_h = sum_j p_j l_j. */
+ORC_API int orc_latent_attend(const uint8_t* ldata, const uint8_t* lscale, int64_t cap, const uint8_t* swa,
+                              int64_t swa_cap, int64_t qpos, const uint16_t* q /*[hq][512]*/, int hq,
+                              const int32_t* idx, int k, int64_t swa_begin, int win, double sm_scale,
+                              double* out /*[hq][512]*/, double* lse /*[hq]*/, int ratio)
+{
+    const int64_t vis = orc_visible(qpos, ratio);
+    int64_t lo = qpos - win + 1;
+    if (lo < swa_begin) lo = swa_begin;
+    if (lo < 0) lo = 0;
+    int nw = (int)(qpos - lo + 1);
+    if (nw < 0) nw = 0;
+    double* L = (double*)malloc(sizeof(double) * 512 * (k + nw + 1));
+    int nk = 0;
+    for (int j = 0; j < k; ++j) {
+        if (idx[j] < 0) continue;
+        if (idx[j] >= vis || idx[j] >= cap) { free(L); return -1; }
+        orc_dequant_rows(ldata + (int64_t)idx[j] * 256, lscale + (int64_t)idx[j] * 32, 1, 512, L + nk * 512);
+        ++nk;
+    }
+    for (int64_t p = lo; p <= qpos; ++p) {
+        const uint8_t* e = swa + (p & (swa_cap - 1)) * 512;
+        for (int d = 0; d < 512; ++d) L[nk * 512 + d] = orc_e4m3_decode(e[d]);
+        ++nk;
+    }
+    double* lg = (double*)malloc(sizeof(double) * (nk + 1));
+    for (int h = 0; h < hq; ++h) {
+        double m = -INFINITY, l = 0.0;
+        for (int j = 0; j < nk; ++j) {
+            double dot = 0.0;
+            for (int d = 0; d < 512; ++d) dot += bf16_to_double(q[h * 512 + d]) * L[j * 512 + d];
+            lg[j] = dot * sm_scale;
+            if (lg[j] > m) m = lg[j];
+        }
+        for (int d = 0; d < 512; ++d) out[h * 512 + d] = 0.0;
+        for (int j = 0; j < nk; ++j) {
+            double pj = exp(lg[j] - m);
+            l += pj;
+            for (int d = 0; d < 512; ++d) out[h * 512 + d] += pj * L[j * 512 + d];
+        }
+        for (int d = 0; d < 512; ++d) out[h * 512 + d] = (nk > 0) ? out[h * 512 + d] / l : 0.0;
+        lse[h] = (nk > 0) ? m + log(l) : -INFINITY;
+    }
+    free(L); free(lg);
     return nk;
 }

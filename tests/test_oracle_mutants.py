@@ -22,6 +22,7 @@ SRC = os.path.join(ROOT, "oracle", "csa2_oracle.c")
 CODEC = ["tests/test_oracle_codec.py", "tests/test_golden_bytes.py"]
 SELECT = ["tests/test_oracle_select.py"]
 ATTN = ["tests/test_oracle_attention.py"]
+PAGES = ["tests/test_oracle_pages_shapes.py"]
 
 # id, text in csa2_oracle.c (must occur exactly once), the planted mistake, pin files that must catch it
 MUTANTS = [
@@ -37,9 +38,11 @@ MUTANTS = [
     ("dequant_scale_block_32", "orc_e4m3_decode(scale[r * nb + c / 16]);", "orc_e4m3_decode(scale[r * nb + c / 32]);",
      CODEC),
     ("entry_bytes_scale_per_32", "return ch / 2 + ch / 16;", "return ch / 2 + ch / 32;", CODEC),
-    ("score_drops_last_head", "for (int h = 0; h < hi; ++h) {", "for (int h = 0; h < hi - 1; ++h) {", SELECT),
+    ("score_drops_last_head", "for (int h = 0; h < hi; ++h) {\n        int g = h * hk / hi;",
+     "for (int h = 0; h < hi - 1; ++h) {\n        int g = h * hk / hi;", SELECT),
     ("key_head_interleaved", "int g = h * hk / hi;", "int g = h % hk;", SELECT),
-    ("relu_ignored", "total += (relu && dot < 0.0) ? 0.0 : dot;", "total += dot;", SELECT),
+    ("relu_ignored", "dot += qd[h * 64 + c] * kv[c];\n        total += (relu && dot < 0.0) ? 0.0 : dot;",
+     "dot += qd[h * 64 + c] * kv[c];\n        total += dot;", SELECT),
     ("query_not_quantised", "orc_dequant_rows(qdata, qscale, hi, 64, qd);",
      "for (int i = 0; i < hi * 64; ++i) qd[i] = bf16_to_double(idx_q[i]);", SELECT),
     ("topk_ties_to_higher_position", "return (x->p < y->p) ? -1 : (x->p > y->p);",
@@ -50,14 +53,39 @@ MUTANTS = [
     ("query_token_not_visible", "return qpos < 0 ? 0 : (qpos + 1) / ratio;", "return qpos < 0 ? 0 : qpos / ratio;",
      SELECT + ATTN),
     ("reindex_ignores_causality", "if (q < vis) p[n++] = q;", "p[n++] = q;", SELECT),
-    ("window_one_key_short", "int64_t lo = qpos - win + 1;", "int64_t lo = qpos - win + 2;", ATTN),
+    ("window_one_key_short", "must be visible (R12) */\n    int64_t lo = qpos - win + 1;",
+     "must be visible (R12) */\n    int64_t lo = qpos - win + 2;", ATTN),
     ("main_v_from_k_half", "memcpy(V + nk * 128, row + 128, 128 * sizeof(double));",
      "memcpy(V + nk * 128, row, 128 * sizeof(double));", ATTN),
     ("window_v_from_k_half", "V[nk * 128 + d] = orc_e4m3_decode(e[128 + d]);",
      "V[nk * 128 + d] = orc_e4m3_decode(e[d]);", ATTN),
-    ("lse_without_max", "lse[h] = (nk > 0) ? m + log(l) : -INFINITY;", "lse[h] = (nk > 0) ? log(l) : -INFINITY;", ATTN),
-    ("attention_skips_last_selected", "for (int j = 0; j < k; ++j) {\n        if (idx[j] < 0) continue;",
-     "for (int j = 0; j < k - 1; ++j) {\n        if (idx[j] < 0) continue;", ATTN),
+    ("lse_without_max", "out[h * 128 + d] / l : 0.0;\n        lse[h] = (nk > 0) ? m + log(l) : -INFINITY;",
+     "out[h * 128 + d] / l : 0.0;\n        lse[h] = (nk > 0) ? log(l) : -INFINITY;", ATTN),
+    ("attention_skips_last_selected", "for (int j = 0; j < k; ++j) {\n        if (idx[j] < 0) continue;\n"
+     "        if (idx[j] >= vis || idx[j] >= c->cap)", "for (int j = 0; j < k - 1; ++j) {\n        if (idx[j] < 0) "
+     "continue;\n        if (idx[j] >= vis || idx[j] >= c->cap)", ATTN),
+    # the pages' own shapes: MXFP4 indexer key, 32 x 128 MQA indexer, 512-channel latent attention
+    ("mx_scale_exponent_off_by_one", "sbyte = (e2 - 1) - 2 + 127;", "sbyte = (e2 - 1) - 1 + 127;", PAGES),
+    ("mx_zero_block_scale_one", "int sbyte = 0;\n            if (amax > 0.0) {",
+     "int sbyte = 127;\n            if (amax > 0.0) {", PAGES),
+    ("mx_nibbles_swapped", "data[r * (ch / 2) + 16 * b + i / 2] = (uint8_t)(c0 | (c1 << 4));",
+     "data[r * (ch / 2) + 16 * b + i / 2] = (uint8_t)(c1 | (c0 << 4));", PAGES),
+    ("mx_scale_read_as_e4m3", "orc_e2m1_decode(code) * orc_e8m0_decode(scale[r * nb + c / 32]);",
+     "orc_e2m1_decode(code) * orc_e4m3_decode(scale[r * nb + c / 32]);", PAGES),
+    ("mx_entry_bytes_scale_per_16", "return ch / 2 + ch / 32;", "return ch / 2 + ch / 16;", PAGES),
+    ("mx_query_not_quantised", "orc_mx_dequant_rows(qdata, qscale, hi, 128, qd);",
+     "for (int i = 0; i < hi * 128; ++i) qd[i] = bf16_to_double(idx_q[i]);", PAGES),
+    ("mx_relu_ignored", "dot += qd[h * 128 + c] * kd[c];\n            total += (relu && dot < 0.0) ? 0.0 : dot;",
+     "dot += qd[h * 128 + c] * kd[c];\n            total += dot;", PAGES),
+    ("latent_window_one_key_short", "const int64_t vis = orc_visible(qpos, ratio);\n    int64_t lo = qpos - win + 1;",
+     "const int64_t vis = orc_visible(qpos, ratio);\n    int64_t lo = qpos - win + 2;", PAGES),
+    ("latent_skips_last_selected", "for (int j = 0; j < k; ++j) {\n        if (idx[j] < 0) continue;\n"
+     "        if (idx[j] >= vis || idx[j] >= cap)", "for (int j = 0; j < k - 1; ++j) {\n        if (idx[j] < 0) "
+     "continue;\n        if (idx[j] >= vis || idx[j] >= cap)", PAGES),
+    ("latent_window_channels_swapped", "L[nk * 512 + d] = orc_e4m3_decode(e[d]);",
+     "L[nk * 512 + d] = orc_e4m3_decode(e[d ^ 1]);", PAGES),
+    ("latent_lse_without_max", "out[h * 512 + d] / l : 0.0;\n        lse[h] = (nk > 0) ? m + log(l) : -INFINITY;",
+     "out[h * 512 + d] / l : 0.0;\n        lse[h] = (nk > 0) ? log(l) : -INFINITY;", PAGES),
 ]
 
 
@@ -90,7 +118,7 @@ def outcomes():
         src = f.read()
     res = {}
     with tempfile.TemporaryDirectory() as d:
-        jobs = {"control": (src, CODEC + SELECT + ATTN)}
+        jobs = {"control": (src, CODEC + SELECT + ATTN + PAGES)}
         for mid, old, new, files in MUTANTS:
             n = src.count(old)
             if n != 1:
