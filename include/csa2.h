@@ -191,8 +191,8 @@ CSA2_API csa2_status csa2_index_topk_reindex(const csa2_shape* shape, const csa2
  *   log) may be NULL.
  * Reading taken here: ONE softmax over selected rows and window rows together; a position may
  * appear in both (its FP4 main entry and its FP8 window entry are different vectors). An index
- * < -1, not visible at qpos (see ratio) or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row with no key gives out = 0
- * and lse = -inf.
+ * < -1, not visible at qpos (see ratio) or >= cap sets CSA2_DEV_BAD_INDEX and is skipped. A row
+ * with no key gives out = 0 and lse = -inf.
  */
 CSA2_API csa2_status csa2_sparse_attend(const csa2_shape* shape, const csa2_cache* cache, int batch, int tq,
                                const int64_t* qpos, const uint16_t* q, const int32_t* idx, int k,
@@ -210,6 +210,10 @@ CSA2_API csa2_status csa2_sparse_attend(const csa2_shape* shape, const csa2_cach
  *                    caller appends it and calls the index step and attention itself)
  *   decode_reindex : appends swa_kv; Reindex index step; attention
  *   decode_minimal : appends swa_kv; attention with the inherited idx
+ * Multi-token decode (t draft tokens per sequence verified together) has no composed call: it is
+ * csa2_quantize_append with t tokens at pos[b], csa2_index_topk_full with tq = t (row i of
+ * sequence b at qpos[b*t + i] = pos[b] + i, no pool) and csa2_sparse_attend with tq = t; the
+ * window ring then needs swa_cap >= win + t.
  */
 CSA2_API csa2_status csa2_decode_full(const csa2_shape* shape, const csa2_cache* cache, int batch, const int64_t* qpos,
                              const uint16_t* kv, const uint16_t* idx_k, const uint16_t* swa_kv,
