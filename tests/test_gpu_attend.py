@@ -1,17 +1,16 @@
 """Sparse attention and the four per-mode compositions on the GPU against the oracle.
 
 Attention outputs (fp32) must be within 2e-3 at unit-variance inputs, scaled with sigma (the bound
-of fp16 products of exact dequantised values with fp32 accumulation); the bf16 output must be the round-to-nearest-even of the fp32 output;
-index outputs of the compositions must be identical to the oracle's.
+of fp16 products of exact dequantised values with fp32 accumulation); the bf16 output must be the
+round-to-nearest-even of the fp32 output; index outputs of the compositions must be identical to the oracle's.
 """
 import numpy as np
 import pytest
 import torch
 
 import compressed_sparse_attention_append_b200 as csa
-import oracle
 import workloads as W
-from _gpu import DEV, attn_tol, bf16_np, gpu_fill, oracle_seq, query_values, values
+from _gpu import DEV, attn_tol, gpu_fill, oracle_seq, query_values, values
 
 pytestmark = pytest.mark.gpu
 

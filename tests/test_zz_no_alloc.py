@@ -6,7 +6,6 @@ workspace, within the attention tolerance. The second call checks that the share
 ready (split tickets back at zero). This file is collected last so that a failure here never hides
 the other tests; it passes alone in a fresh process too.
 """
-import numpy as np
 import pytest
 import torch
 
