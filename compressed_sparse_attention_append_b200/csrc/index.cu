@@ -14,7 +14,7 @@
 //     the positive channels and one prmt of the sign-flipped codes those of the negative ones;
 //   * a 16-channel block's dot product D = sum (2q)(2k) comes from dp4a (|D| <= 2304);
 //   * an E4M3 scale s = M * 2^(E-10) (M <= 15, E >= 1) enters as the integer f(s) = M * 2^(E-1)
-//     (<= 245760); D * f(s_k) fits in int32 and (D * f(s_k)) * f(s_q) is added to an int64
+//     (<= 448 * 2^9 = 229376); D * f(s_k) fits in int32 and (D * f(s_k)) * f(s_q) is added to an int64
 //     with one wide multiply-add (each term < 2^47, the sum of 16 terms < 2^51).
 // No floating-point conversion runs in the scoring loop. Ranking is by S descending, ties to the
 // lower position; S is the same integer the exact rational score gives, so the selected set is
