@@ -126,7 +126,7 @@ CSA2_API csa2_status csa2_workspace_init(void* ws, size_t ws_bytes, void* stream
 
 /*
  * Quantise-append. [C] sec. XI: cached values are E2M1 with one E4M3 scale per 16 channels and
- * no second-level global scale, quantised after RoPE; the sliding-window KV stays at FP8.
+ * no scale for the whole tensor on top, quantised after RoPE; the sliding-window KV stays at FP8.
  * [B] "Technical Approach": Full mode writes main KV and indexer keys, Reindex and Minimal
  * write only their own sliding-window KV (pass NULL for the planes a mode does not write).
  *   pos    [batch] int64 : first new position of each sequence; tokens go to pos..pos+t-1

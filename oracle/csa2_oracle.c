@@ -67,7 +67,7 @@
 
 /* ------------------------------------------------------------------------------------ */
 /* Element formats. [A] last-but-one caption; [C] sec. XI "FP4 Main KV Cache": E2M1 elements, */
-/* one E4M3 scale per 16 channels, no second-level global scale; SWA KV kept at FP8.       */
+/* one E4M3 scale per 16 channels, no tensor-wide scale on top; SWA KV kept at FP8.        */
 /* ------------------------------------------------------------------------------------ */
 
 /* E2M1: sign bit 3, exponent bits 2..1 (bias 1), mantissa bit 0. No inf/NaN. */
