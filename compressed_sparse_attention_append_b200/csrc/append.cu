@@ -1,8 +1,8 @@
 // append.cu -- quantise-append of new tokens into the FP4 cache planes and the FP8 window ring.
 //
 // [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token", sec. XI:
-// E2M1 elements with one E4M3 scale per 16 channels and no scale for the whole tensor on top, quantised
-// after RoPE; the sliding-window KV stays at FP8. [B] "DeepSeek Cuts KV Cache Footprint
+// E2M1 elements with one E4M3 scale per 16 channels and no scale for the whole tensor on top,
+// quantised after RoPE; the sliding-window KV stays at FP8. [B] "DeepSeek Cuts KV Cache Footprint
 // Fourfold", "Technical Approach": only Full mode writes main KV and indexer keys; every mode
 // writes its own sliding-window KV.
 //
