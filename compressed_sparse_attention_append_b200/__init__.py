@@ -123,6 +123,28 @@ def _p(t):
     return t.data_ptr()
 
 
+def _typed(t, dtype):
+    if t is None:
+        return None
+    assert isinstance(t, torch.Tensor) and t.dtype == dtype, f"expected a {dtype} tensor"
+    return _p(t)
+
+
+def _i64(t):
+    """int64 arrays of include/csa2.h (positions): pointer only, after a dtype check."""
+    return _typed(t, torch.int64)
+
+
+def _i32(t):
+    """int32 arrays of include/csa2.h (indices, pools, counts): pointer only, after a dtype check."""
+    return _typed(t, torch.int32)
+
+
+def _f32(t):
+    """fp32 outputs of include/csa2.h (out_f32, lse): pointer only, after a dtype check."""
+    return _typed(t, torch.float32)
+
+
 def _bits(t):
     """bf16 tensors travel as their 16-bit patterns; pointer only."""
     if t is None:
@@ -204,7 +226,7 @@ class Workspace:
 
 def csa2_quantize_append(shape, cache: Cache, batch, t, pos, kv=None, idx_k=None, swa_kv=None, ws=None, stream=None):
     _check("csa2_quantize_append", lib().csa2_quantize_append(
-        ctypes.byref(shape), cache.ref, batch, t, _p(pos), _bits(kv), _bits(idx_k), _bits(swa_kv),
+        ctypes.byref(shape), cache.ref, batch, t, _i64(pos), _bits(kv), _bits(idx_k), _bits(swa_kv),
         ws.ptr if ws else None, ws.nbytes if ws else 0, _stream(stream)))
 
 
@@ -213,30 +235,30 @@ def csa2_index_topk_full(shape, cache: Cache, batch, tq, qpos, idx_q, k, out_idx
     if max_ctx is None:
         max_ctx = cache.cap
     _check("csa2_index_topk_full", lib().csa2_index_topk_full(
-        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(idx_q), k, _p(out_idx), pool_blocks, _p(out_pool),
-        _p(out_pool_n), max_ctx, flags, ws.ptr, ws.nbytes, _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, tq, _i64(qpos), _bits(idx_q), k, _i32(out_idx), pool_blocks, _i32(out_pool),
+        _i32(out_pool_n), max_ctx, flags, ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_index_topk_reindex(shape, cache: Cache, batch, qpos, idx_q, pool, pool_n, k, out_idx, flags=0, ws=None,
                             stream=None):
     _check("csa2_index_topk_reindex", lib().csa2_index_topk_reindex(
-        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(idx_q), _p(pool), _p(pool_n), pool.shape[-1], k,
-        _p(out_idx), flags, ws.ptr, ws.nbytes, _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, _i64(qpos), _bits(idx_q), _i32(pool), _i32(pool_n), pool.shape[-1], k,
+        _i32(out_idx), flags, ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_sparse_attend(shape, cache: Cache, batch, tq, qpos, q, idx, k, out, swa_begin=None, sm_scale=0.0,
                        out_f32=None, lse=None, ws=None, stream=None):
     _check("csa2_sparse_attend", lib().csa2_sparse_attend(
-        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
-        _bits(out), _p(out_f32), _p(lse), ws.ptr, ws.nbytes, _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, tq, _i64(qpos), _bits(q), _i32(idx), k, _i64(swa_begin), sm_scale,
+        _bits(out), _f32(out_f32), _f32(lse), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_sparse_attend_noalloc(shape, cache: Cache, batch, tq, qpos, q, idx, k, out, swa_begin=None, sm_scale=0.0,
                                out_f32=None, lse=None, stream=None):
     """csa2_sparse_attend without a workspace (scratch in a static device array inside libcsa2)."""
     _check("csa2_sparse_attend_noalloc", lib().csa2_sparse_attend_noalloc(
-        ctypes.byref(shape), cache.ref, batch, tq, _p(qpos), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
-        _bits(out), _p(out_f32), _p(lse), _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, tq, _i64(qpos), _bits(q), _i32(idx), k, _i64(swa_begin), sm_scale,
+        _bits(out), _f32(out_f32), _f32(lse), _stream(stream)))
 
 
 def csa2_decode_full(shape, cache: Cache, batch, qpos, kv, idx_k, swa_kv, idx_q, q, k, out_idx, out, pool_blocks=0,
@@ -245,31 +267,31 @@ def csa2_decode_full(shape, cache: Cache, batch, qpos, kv, idx_k, swa_kv, idx_q,
     if max_ctx is None:
         max_ctx = cache.cap
     _check("csa2_decode_full", lib().csa2_decode_full(
-        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(kv), _bits(idx_k), _bits(swa_kv), _bits(idx_q),
-        _bits(q), k, _p(out_idx), pool_blocks, _p(out_pool), _p(out_pool_n), max_ctx, _p(swa_begin), sm_scale,
-        _bits(out), _p(out_f32), _p(lse), flags, ws.ptr, ws.nbytes, _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, _i64(qpos), _bits(kv), _bits(idx_k), _bits(swa_kv), _bits(idx_q),
+        _bits(q), k, _i32(out_idx), pool_blocks, _i32(out_pool), _i32(out_pool_n), max_ctx, _i64(swa_begin), sm_scale,
+        _bits(out), _f32(out_f32), _f32(lse), flags, ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_decode_reindex(shape, cache: Cache, batch, qpos, swa_kv, idx_q, q, pool, pool_n, k, out_idx, out,
                         swa_begin=None, sm_scale=0.0, out_f32=None, lse=None, flags=0, ws=None, stream=None):
     _check("csa2_decode_reindex", lib().csa2_decode_reindex(
-        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(swa_kv), _bits(idx_q), _bits(q), _p(pool), _p(pool_n),
-        pool.shape[-1], k, _p(out_idx), _p(swa_begin), sm_scale, _bits(out), _p(out_f32), _p(lse), flags, ws.ptr,
+        ctypes.byref(shape), cache.ref, batch, _i64(qpos), _bits(swa_kv), _bits(idx_q), _bits(q), _i32(pool), _i32(pool_n),
+        pool.shape[-1], k, _i32(out_idx), _i64(swa_begin), sm_scale, _bits(out), _f32(out_f32), _f32(lse), flags, ws.ptr,
         ws.nbytes, _stream(stream)))
 
 
 def csa2_decode_minimal(shape, cache: Cache, batch, qpos, swa_kv, q, idx, k, out, swa_begin=None, sm_scale=0.0,
                         out_f32=None, lse=None, ws=None, stream=None):
     _check("csa2_decode_minimal", lib().csa2_decode_minimal(
-        ctypes.byref(shape), cache.ref, batch, _p(qpos), _bits(swa_kv), _bits(q), _p(idx), k, _p(swa_begin), sm_scale,
-        _bits(out), _p(out_f32), _p(lse), ws.ptr, ws.nbytes, _stream(stream)))
+        ctypes.byref(shape), cache.ref, batch, _i64(qpos), _bits(swa_kv), _bits(q), _i32(idx), k, _i64(swa_begin), sm_scale,
+        _bits(out), _f32(out_f32), _f32(lse), ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_prefill_chunk(shape, cache: Cache, pos0, t, kv, idx_k, swa_kv, idx_q, q, k, out_idx, out, swa_begin=0,
                        sm_scale=0.0, out_f32=None, lse=None, flags=0, ws=None, stream=None):
     _check("csa2_prefill_chunk", lib().csa2_prefill_chunk(
         ctypes.byref(shape), cache.ref, pos0, t, _bits(kv), _bits(idx_k), _bits(swa_kv), _bits(idx_q), _bits(q), k,
-        _p(out_idx), swa_begin, sm_scale, _bits(out), _p(out_f32), _p(lse), flags, ws.ptr, ws.nbytes,
+        _i32(out_idx), swa_begin, sm_scale, _bits(out), _f32(out_f32), _f32(lse), flags, ws.ptr, ws.nbytes,
         _stream(stream)))
 
 

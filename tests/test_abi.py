@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import compressed_sparse_attention_append_b200 as csa
 from conftest import ROOT
@@ -199,3 +200,27 @@ def test_product_path_has_no_oracle_dependency():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 txt = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in txt.lower(), f
+
+
+def test_binding_checks_integer_and_float_dtypes(L):
+    """The binding refuses an array of the wrong dtype before anything reaches the library (a kernel
+    would read an int32 array as int64, or the reverse); the dtype check runs before the device check,
+    so CPU tensors show it here."""
+    import types
+
+    shape = csa.make_shape()
+    cache = types.SimpleNamespace(ref=ctypes.byref(csa.csa2_cache()), cap=64)  # never dereferenced here
+    swa = torch.zeros(1, 1, 256, dtype=torch.bfloat16)
+    with pytest.raises(AssertionError, match="int64"):
+        csa.csa2_quantize_append(shape, cache, 1, 1, torch.zeros(1, dtype=torch.int32), swa_kv=swa)
+    with pytest.raises(AssertionError, match="int64"):
+        csa.csa2_sparse_attend(shape, cache, 1, 1, torch.zeros(1, dtype=torch.int32), None, None, 512, None)
+    with pytest.raises(AssertionError, match="CUDA"):  # right dtype: the device check comes next
+        csa.csa2_quantize_append(shape, cache, 1, 1, torch.zeros(1, dtype=torch.int64), swa_kv=swa)
+    for fn, good, bad in ((csa._i32, torch.int32, torch.int64), (csa._i64, torch.int64, torch.int32),
+                          (csa._f32, torch.float32, torch.bfloat16)):
+        with pytest.raises(AssertionError, match=str(good)):
+            fn(torch.zeros(2, dtype=bad))
+        with pytest.raises(AssertionError, match="CUDA"):
+            fn(torch.zeros(2, dtype=good))
+        assert fn(None) is None
