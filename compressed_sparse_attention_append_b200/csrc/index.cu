@@ -1,6 +1,7 @@
 // index.cu -- indexer scoring and exact Top-k selection for several query rows per sequence (the
-// prefill chunk: row i of a chunk sees positions <= i). Rows of one query per sequence (decode:
-// Full with its block pool, and Reindex) run in index_decode.cu.
+// prefill chunk, where row i of a chunk sees positions <= i, and multi-token decode, where the
+// draft tokens of a sequence are verified together). Rows of one query per sequence (decode: Full
+// with its block pool, and Reindex) run in index_decode.cu.
 //
 // [B] "DeepSeek Cuts KV Cache Footprint Fourfold", "Technical Approach": Full mode computes the
 // Top-K indices. [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token",
