@@ -28,6 +28,11 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 // Device address of the array on each device, taken once with that device current. A host-side
 // reference to g_noalloc_scratch names a host stand-in, never the device memory itself.
+// The array needs no clearing: a __device__ array without an initialiser is zero when the module
+// is loaded on a device, and every call leaves the tickets it used at zero again. (Clearing it here
+// with a memset would need ordering against the caller's stream, which may be a non-blocking one.)
+// The cached address belongs to the device's primary context: after cudaDeviceReset the module is
+// loaded afresh at another address, so this entry point must not be used after a device reset.
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[256] = {};
 
@@ -38,8 +43,6 @@ csa2_status noalloc_scratch(void** out) {
     if (!g_noalloc_ptr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return CSA2_ERR_CUDA;
-        // counters must start at zero; every call leaves them at zero again
-        if (cudaMemset(p, 0, kNoAllocBytes) != cudaSuccess) return CSA2_ERR_CUDA;
         g_noalloc_ptr[dev] = p;
     }
     *out = g_noalloc_ptr[dev];

@@ -257,8 +257,10 @@ CSA2_API csa2_status csa2_prefill_chunk(const csa2_shape* shape, const csa2_cach
  * device.
  *   - Scratch: a 4 MiB file-scope device array per GPU, held until the process exits.
  *   - Limit: batch * tq <= 1024; larger calls return CSA2_ERR_CAPACITY.
- *   - The first call on a device takes the array's device address (cudaGetSymbolAddress) and
- *     zeroes it with a synchronous cudaMemset; make that first call before any stream capture.
+ *   - The array is zero when the library's module is loaded on a device, and every call leaves
+ *     its split tickets at zero again, so no clearing is needed. The first call on a device takes
+ *     the array's device address (cudaGetSymbolAddress) and keeps it; make that first call before
+ *     any stream capture, and do not call this entry point after cudaDeviceReset on that device.
  *   - Every call shares the one array: calls whose kernels overlap on the GPU (other streams,
  *     other threads) race and must be serialised by the caller.
  *   - Device-side status bits (bad indices) are not reported; bad indices are still skipped.

@@ -309,10 +309,9 @@ ORC_API int orc_topk(const double* scores, const int64_t* pos, int64_t n, int k,
     return m;
 }
 
-/* Block pool (R10). [C] sec. VI "Shortlist-of-a-shortlist" and sec. IX Figure 4: each
- * block of `bs` positions is scored by the maximum index score among its (visible)
- * positions; the winning blocks form the candidate pool, up to `pool_blocks` (2,048) of
- * them. Blocks rank by block score descending, ties to the lower block id; the pool is
+/* Block pool (R10). [C] sec. VI "Shortlist-of-a-shortlist" and sec. IX Figure 4: a block's
+ * score is the largest score of its visible positions (`bs` positions per block), and the
+ * best blocks, at most `pool_blocks` (2,048) of them, make up the candidate pool. Blocks rank by block score descending, ties to the lower block id; the pool is
  * emitted as ascending block ids. scores[p] for p in [0, n). */
 ORC_API int orc_pool(const double* scores, int64_t n, int bs, int pool_blocks, int32_t* out)
 {
