@@ -41,6 +41,7 @@ CSA2_ERR_DEVICE = 6
 CSA2_DEV_BAD_INDEX = 0x1
 CSA2_DEV_BAD_POS = 0x2
 CSA2_DEV_BAD_POOL = 0x4
+CSA2_DEV_TIMEOUT = 0x8
 CSA2_SCORE_RELU = 0x1
 
 EXPORTS = (

@@ -20,56 +20,6 @@ namespace csa2 {
 
 namespace {
 
-// Two fp32 -> one byte of two E2M1 codes (first argument -> low nibble), RNE, saturating.
-__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
-    uint16_t r;
-    asm("{\n\t.reg .b8 t;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
-        "mov.b16 %0, {t, 0};\n\t}"
-        : "=h"(r)
-        : "f"(lo), "f"(hi));
-    return r & 0xFF;
-}
-
-// Two fp32 -> two E4M3 bytes (first argument -> low byte), RNE, saturating to +-448.
-__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
-    uint16_t r;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&x)[16]) {
-    uint4 a = *reinterpret_cast<const uint4*>(p);
-    uint4 b = *reinterpret_cast<const uint4*>(p + 8);
-    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-
-// One 16-channel block: 8 code bytes + 1 scale byte.
-__device__ __forceinline__ void quantize_block(const float (&x)[16], uint2& codes, uint8_t& scale) {
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
-    float s32 = __fdiv_rn(amax, 6.0f);
-    uint32_t sc = f32x2_to_e4m3x2(s32, 0.f) & 0xFF;
-    float s = e4m3_to_f32((uint8_t)sc);
-    uint32_t b[8];
-    if (s == 0.f) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) b[j] = 0;
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) b[j] = f32x2_to_e2m1x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
-    }
-    codes.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-    codes.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
-    scale = (uint8_t)sc;
-}
-
 __global__ void __launch_bounds__(192) append_kernel(AppendArgs a) {
     // the slots written here may still be read by the previous step's attention (the window ring)
     wait_prior_grid();

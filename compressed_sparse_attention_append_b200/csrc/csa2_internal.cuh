@@ -31,6 +31,8 @@ constexpr int kBS = 8;        // positions per pool block
 constexpr int kSWABytes = 256;
 constexpr int kMaxK = 2048;   // largest Top-k / pool size
 constexpr int kPartStride = kD + 4;  // floats per (split, head) partial: O[128], m, l, 2 pad (16-byte rows)
+constexpr int kKeyBins = 2048;  // score histogram bins of a decode row (sign, exponent, 4 mantissa bits)
+constexpr int kSubBins = 1024;  // second-level bins (the next 10 bits) of a decode row's cut bin
 
 // ---- device status word (first 4 bytes of the workspace) --------------------------------------
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t bit) {
@@ -92,6 +94,77 @@ __device__ __forceinline__ uint64_t score_key(double s) {
     return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
+// ---- codec: quantise one 16-channel block (the rule of include/csa2.h) -----------------------
+// Two fp32 -> one byte of two E2M1 codes (first argument -> low nibble), RNE, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\t"
+        "mov.b16 %0, {t, 0};\n\t}"
+        : "=h"(r)
+        : "f"(lo), "f"(hi));
+    return r & 0xFF;
+}
+
+// Two fp32 -> two E4M3 bytes (first argument -> low byte), RNE, saturating to +-448.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void load16_bf16(const uint16_t* p, float (&x)[16]) {
+    uint4 a = *reinterpret_cast<const uint4*>(p);
+    uint4 b = *reinterpret_cast<const uint4*>(p + 8);
+    uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// One 16-channel block: 8 code bytes + 1 scale byte.
+__device__ __forceinline__ void quantize_block(const float (&x)[16], uint2& codes, uint8_t& scale) {
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    float s32 = __fdiv_rn(amax, 6.0f);
+    uint32_t sc = f32x2_to_e4m3x2(s32, 0.f) & 0xFF;
+    float s = e4m3_to_f32((uint8_t)sc);
+    uint32_t b[8];
+    if (s == 0.f) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = 0;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) b[j] = f32x2_to_e2m1x2(__fdiv_rn(x[2 * j], s), __fdiv_rn(x[2 * j + 1], s));
+    }
+    codes.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+    codes.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+    scale = (uint8_t)sc;
+}
+
+// ---- score keys and their histogram bins ----------------------------------------------------------
+// Histogram bin of an orderable score key (0 = no key): the score rounded to fp32 (round to
+// nearest, so a larger score never rounds lower), then its sign, exponent and the top 4 mantissa
+// bits. A larger key never has a smaller bin. Nonzero scores (|score| < 2^51) have exponents
+// 127..178, so the positive bins are 1024 + 16..847 and the negative ones mirror them below 1024.
+__device__ __forceinline__ int key_bin(unsigned long long key) {
+    const unsigned int b = __float_as_uint(__ll2float_rn((long long)(key ^ 0x8000000000000000ull)));
+    const int em = (int)((b >> 19) & 0xFFFu);  // exponent * 16 + top 4 mantissa bits
+    const int f = em ? em - (126 << 4) : 0;
+    return (b >> 31) ? kKeyBins / 2 - 1 - f : kKeyBins / 2 + f;
+}
+
+// Second-level bin of a key inside its key_bin: the next 10 mantissa bits of the same fp32 value,
+// ordered like the keys within the bin.
+__device__ __forceinline__ int sub_bin(unsigned long long key) {
+    const unsigned int b = __float_as_uint(__ll2float_rn((long long)(key ^ 0x8000000000000000ull)));
+    const int sb = (int)((b >> 9) & (unsigned int)(kSubBins - 1));
+    return (b >> 31) ? kSubBins - 1 - sb : sb;
+}
+
 // ---- programmatic dependent launch -----------------------------------------------------------------
 // Kernels that read an earlier kernel's output are launched with programmatic stream serialisation,
 // so that their launch overlaps the end of the kernel before them; each one waits here before its
@@ -143,9 +216,11 @@ struct IndexPlan {
 
 struct AttendPlan {
     int rows;
-    int nk_max;        // k + win
-    int kps;           // keys per split (multiple of 64)
+    int tiles;         // key tiles of a row: ceil(k / 16) tiles of selected entries, then ceil(win / 8) of the window
+    int tps;           // tiles per split
     int splits;
+    int warps;         // warps per CTA: 16 (one CTA per SM) or 8 (two CTAs per SM)
+    int stages;        // gather ring depth per warp (3 with 16 warps, 5 with 8)
 };
 
 // Workspace: a fixed counter area first (its offsets never depend on the call, so counters
@@ -155,9 +230,7 @@ struct AttendPlan {
 //   [.., +4*kMaxRows)   attention ticket per row
 //   data: candidates, block maxima, attention partials (contents are scratch)
 constexpr int kMaxRows = 65536;
-constexpr int kKeyBins = 2048;  // score histogram bins of a decode row (sign, exponent, 4 mantissa bits)
 constexpr int kSelCand = 4096;  // candidates of a decode row ranked by its last select CTA
-constexpr int kSubBins = 1024;  // second-level bins (the next 10 bits) of a decode row's cut bin
 // per decode row: key histogram, block-maximum histogram, and the two second-level histograms
 constexpr int kRowHist = 2 * (kKeyBins + kSubBins);
 constexpr size_t kHdrStatus = 0, kHdrIndexNext = 8, kHdrIndexDone = 12;
@@ -209,18 +282,23 @@ inline IndexPlan make_index_plan(int rows, int tq, int k, int64_t max_scan, int 
 }
 
 inline AttendPlan make_attend_plan(int rows, int k, int win) {
-    // CTAs of 8 warps, two per SM: about 296 CTAs in flight; a split covers at least 256 keys
-    // (two 16-key tiles per warp) so that each warp keeps tiles in flight
+    // A row's key tiles (16 selected entries, or 8 window rows, each) are split over the warps of one
+    // CTA; 16 warps run on every SM (one CTA of 16 warps, or two of 8 when there are more CTAs than
+    // SMs). Large batches take one CTA per row; small ones split a row's tiles over several CTAs (at
+    // least one tile per warp each) so that about one CTA runs per SM, and merge the splits through
+    // the workspace.
     AttendPlan a{};
     a.rows = rows;
-    a.nk_max = k + win;
-    const int units = (a.nk_max + 127) / 128;  // 128 keys = one tile per warp
-    int max_splits = units / 2 > 1 ? units / 2 : 1;
-    int splits = 296 / (rows > 0 ? rows : 1);
+    a.tiles = (k + 15) / 16 + (win + 7) / 8;
+    int max_splits = a.tiles / 16 > 1 ? a.tiles / 16 : 1;
+    int splits = rows >= 74 ? 1 : 148 / (rows > 0 ? rows : 1);
     if (splits < 1) splits = 1;
     if (splits > max_splits) splits = max_splits;
-    a.kps = ((units + splits - 1) / splits) * 128;
-    a.splits = (a.nk_max + a.kps - 1) / a.kps;
+    a.tps = (a.tiles + splits - 1) / splits;
+    a.splits = (a.tiles + a.tps - 1) / a.tps;
+    const bool two_per_sm = (long long)rows * a.splits > 148;
+    a.warps = two_per_sm ? 8 : 16;
+    a.stages = two_per_sm ? 5 : 3;
     return a;
 }
 
@@ -282,6 +360,8 @@ struct IndexArgs {
 };
 cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);         // index.cu: any tq
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s);  // index_decode.cu: plan.decode
+bool index_tc_fits(const IndexPlan& p);                              // index_tc.cu: rows of <= 16,384 positions
+cudaError_t launch_index_tc(const IndexArgs& a, cudaStream_t s);      // index_tc.cu
 
 struct AttendArgs {
     csa2_cache c;

@@ -78,25 +78,6 @@ __device__ __forceinline__ uint32_t e2m1_int2(uint32_t c) {
     return (c & 8) ? ((0u - mag) & 0xFF) : mag;
 }
 
-// Histogram bin of an orderable score key (0 = no key): the score rounded to fp32 (round to
-// nearest, so a larger score never rounds lower), then its sign, exponent and the top 4 mantissa
-// bits. A larger key never has a smaller bin. Nonzero scores (|score| < 2^51) have exponents
-// 127..178, so the positive bins are 1024 + 16..847 and the negative ones mirror them below 1024.
-__device__ __forceinline__ int key_bin(unsigned long long key) {
-    const unsigned int b = __float_as_uint(__ll2float_rn((long long)(key ^ 0x8000000000000000ull)));
-    const int em = (int)((b >> 19) & 0xFFFu);  // exponent * 16 + top 4 mantissa bits
-    const int f = em ? em - (126 << 4) : 0;
-    return (b >> 31) ? kKeyBins / 2 - 1 - f : kKeyBins / 2 + f;
-}
-
-// Second-level bin of a key inside its key_bin: the next 10 mantissa bits of the same fp32 value,
-// ordered like the keys within the bin.
-__device__ __forceinline__ int sub_bin(unsigned long long key) {
-    const unsigned int b = __float_as_uint(__ll2float_rn((long long)(key ^ 0x8000000000000000ull)));
-    const int sb = (int)((b >> 9) & (unsigned int)(kSubBins - 1));
-    return (b >> 31) ? kSubBins - 1 - sb : sb;
-}
-
 struct DRow {
     int64_t qpos;  // the last visible entry: floor((query token + 1) / ratio) - 1
     int b;
@@ -961,6 +942,8 @@ __global__ void zero_kernel(uint4* p, size_t n16) {
 }  // namespace
 
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s) {
+    // rows short enough for one CTA's shared memory: scored on the tensor cores and selected in place
+    if (index_tc_fits(a.plan)) return launch_index_tc(a, s);
     const bool relu = (a.flags & CSA2_SCORE_RELU) != 0;
     const bool pool = a.plan.pool_blocks > 0 && !a.reindex;
     const void* fn = relu ? (pool ? (const void*)score_kernel<true, true> : (const void*)score_kernel<true, false>)

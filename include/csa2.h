@@ -58,6 +58,7 @@ typedef enum {
 #define CSA2_DEV_BAD_INDEX   0x1   /* selected / inherited index < -1, > qpos or >= cap       */
 #define CSA2_DEV_BAD_POS     0x2   /* append position outside [0, cap) or qpos >= bound       */
 #define CSA2_DEV_BAD_POOL    0x4   /* pool block id outside [0, cap / bs)                     */
+#define CSA2_DEV_TIMEOUT     0x8   /* a tensor-core pipeline wait ran out (no output written)  */
 
 /* Flags for the index entry points. */
 #define CSA2_SCORE_RELU      0x1u  /* score = sum_h max(0, q_h . k_h) instead of sum_h q_h . k_h */

@@ -1,20 +1,21 @@
-"""The workloads at full size, in the launch configuration bench.py times, checked on sampled
-sequences (prefill: sampled query rows; multi-token decode: every row of sampled sequences) against
-the oracle: index sets and pools identical, attention within tolerance."""
+"""The workloads at full size, in the launch configuration bench.py times, checked against the
+oracle on every sequence (prefill: 72 query rows spread over the chunk, its first and last rows
+among them; multi-token decode: every row of every sequence): index sets and pools identical,
+attention within tolerance. The oracle runs in spawned host processes."""
 import numpy as np
 import pytest
 import torch
 
-from oracle import workload as OW
+from _oracle_pool import oracle_steps
 from workloads import gpu as G
 
 pytestmark = pytest.mark.gpu
 
 CASES = [
     ("full_b1_n4096", [0]),
-    ("full_b64_n131072", [0, 63]),
-    ("reindex_b128_n1m", [0, 77, 127]),
-    ("minimal_b256_n262144", [0, 100, 255]),
+    ("full_b64_n131072", list(range(64))),
+    ("reindex_b128_n1m", list(range(128))),
+    ("minimal_b256_n262144", list(range(256))),
 ]
 
 
@@ -33,9 +34,9 @@ def test_decode_workload_sampled(orc, name, seqs):
 
     assert csa.csa2_get_device_status(step.ws) == 0
     wl = step.wl
+    ref = oracle_steps(name, seqs)
     for b in seqs:
-        c, inp = OW.build_sequence(wl, b)
-        r = OW.run_step(c, wl, inp)
+        r = ref[b]
         if wl.mode != "minimal":
             assert np.array_equal(step.outputs["idx"][b].cpu().numpy(), r["idx"]), b
         if wl.mode == "full" and wl.pool_blocks:
@@ -58,9 +59,10 @@ def test_prefill_workload_sampled_rows(orc):
     of = torch.empty(wl.tq, 16, 128, dtype=torch.float32, device="cuda")
     step.run(out_f32=of)
     torch.cuda.synchronize()
-    rows = [0, 1, 2047, 4095]
-    c, inp = OW.build_sequence(wl, 0)
-    r = OW.run_step(c, wl, inp, rows=rows)
+    rows = sorted(set([0, 1, 2, 3, 2047, 4094, 4095] + list(range(5, 4096, 63))))
+    assert len(rows) >= 64
+    groups = [rows[j::16] for j in range(16)]
+    r = oracle_steps(name, [0], rows=groups)[0]
     for i in rows:
         idx, ro, _ = r["rows"][i]
         assert np.array_equal(step.outputs["idx"][i].cpu().numpy(), idx), i
@@ -71,7 +73,7 @@ def test_prefill_workload_sampled_rows(orc):
 
 def test_draft_workload_sampled(orc):
     """Multi-token decode (5 draft tokens per sequence, 64 sequences at N = 131,072): the three calls
-    bench.py times; every row of sampled sequences against the oracle."""
+    bench.py times; every row of every sequence against the oracle."""
     import compressed_sparse_attention_append_b200 as csa
 
     step = G.build("draft_b64_n131072_tq5")
@@ -79,9 +81,9 @@ def test_draft_workload_sampled(orc):
     of = torch.empty(step.batch, wl.tq, 16, 128, dtype=torch.float32, device="cuda")
     step.run(out_f32=of)
     assert csa.csa2_get_device_status(step.ws) == 0
-    for b in (0, 63):
-        c, inp = OW.build_sequence(wl, b)
-        r = OW.run_step(c, wl, inp)
+    ref = oracle_steps("draft_b64_n131072_tq5", list(range(step.batch)))
+    for b in range(step.batch):
+        r = ref[b]
         for t in range(wl.tq):
             idx, ro, _ = r["rows"][t]
             assert np.array_equal(step.outputs["idx"][b, t].cpu().numpy(), idx), (b, t)
