@@ -60,20 +60,13 @@ def algorithmic_bytes(wl):
 L2_BYTES = 126 * 1024 * 1024
 
 
-def fused_index(wl):
-    """The decode index step of rows of at most 16,384 positions runs as one tensor-core kernel;
-    longer rows as zero + score + select."""
-    scan = wl.pool_blocks * wl.bs if wl.mode == "reindex" else wl.context
-    return scan <= 16384
-
-
 def kernels_per_step(wl):
-    """Kernels one step launches: append 1; index: 1 (one tensor-core kernel, or the multi-row kernel)
-    or 3 (zero + score + select); attention 1."""
+    """Kernels one step launches: append 1; index: 3 for decode rows (zero + score + select), 1 for
+    several rows per sequence (the multi-row kernel); attention 1."""
     if wl.mode == "minimal":
         return 2
     if wl.mode in ("full", "reindex"):
-        return 3 if fused_index(wl) else 5
+        return 5
     return 3
 
 
@@ -504,9 +497,7 @@ def run_gpu(args):
     else:
         dom_bytes = ab[dom] * B
         # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
-        if dom == "index" and fused_index(wl):
-            dom_file, dom_kernels = "index_tc.cu", "index_tc_kernel"
-        elif dom == "index":
+        if dom == "index":
             dom_file, dom_kernels = "index_decode.cu", "zero_kernel + score_kernel + select_kernel"
         else:
             dom_file, dom_kernels = "attend.cu", "attend_kernel"

@@ -448,7 +448,8 @@ __global__ void __launch_bounds__(W * 32, (W == 8 ? 2 : 1)) attend_kernel(Attend
         if (!s_last || !wr) return;
         __threadfence();
         // the other splits' partials, read from L2 (they were written by other CTAs); this split's
-        // own partial is still in registers
+        // own partial is still in registers. The splits are folded in index order, whichever CTA
+        // finished last, so that the result does not depend on the order the splits finished in.
         const float M_own = M, L_own = Lsum;
         float acc_own[8];
 #pragma unroll
@@ -456,22 +457,27 @@ __global__ void __launch_bounds__(W * 32, (W == 8 ? 2 : 1)) attend_kernel(Attend
         M = M_own;
         for (int sp = 0; sp < splits; ++sp)
             if (sp != split) M = fmaxf(M, __ldcg(part + ((size_t)sp * kHQ + h) * kPartStride + kD));
-        {
-            const float f = (M_own == -INFINITY) ? 0.f : exp2f(M_own - M);
-            Lsum = f * L_own;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] = f * acc_own[j];
-        }
+        Lsum = 0.f;
         for (int sp = 0; sp < splits; ++sp) {
-            if (sp == split) continue;
-            const float* q = part + ((size_t)sp * kHQ + h) * kPartStride;
-            const float4 v0 = __ldcg(reinterpret_cast<const float4*>(q + d0));
-            const float4 v1 = __ldcg(reinterpret_cast<const float4*>(q + d0 + 4));
-            const float mw = __ldcg(q + kD), lw = __ldcg(q + kD + 1);
+            float mw, lw, v[8];
+            if (sp == split) {
+                mw = M_own;
+                lw = L_own;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = acc_own[j];
+            } else {
+                const float* q = part + ((size_t)sp * kHQ + h) * kPartStride;
+                const float4 v0 = __ldcg(reinterpret_cast<const float4*>(q + d0));
+                const float4 v1 = __ldcg(reinterpret_cast<const float4*>(q + d0 + 4));
+                mw = __ldcg(q + kD);
+                lw = __ldcg(q + kD + 1);
+                v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w;
+                v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+            }
             const float f = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
             Lsum += f * lw;
-            acc[0] += f * v0.x; acc[1] += f * v0.y; acc[2] += f * v0.z; acc[3] += f * v0.w;
-            acc[4] += f * v1.x; acc[5] += f * v1.y; acc[6] += f * v1.z; acc[7] += f * v1.w;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] += f * v[j];
         }
         if (tid == 0) *tk = 0;
     }

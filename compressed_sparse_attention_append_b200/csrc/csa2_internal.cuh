@@ -360,8 +360,6 @@ struct IndexArgs {
 };
 cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);         // index.cu: any tq
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s);  // index_decode.cu: plan.decode
-bool index_tc_fits(const IndexPlan& p);                              // index_tc.cu: rows of <= 16,384 positions
-cudaError_t launch_index_tc(const IndexArgs& a, cudaStream_t s);      // index_tc.cu
 
 struct AttendArgs {
     csa2_cache c;

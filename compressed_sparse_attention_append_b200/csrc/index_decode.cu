@@ -942,8 +942,6 @@ __global__ void zero_kernel(uint4* p, size_t n16) {
 }  // namespace
 
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s) {
-    // rows short enough for one CTA's shared memory: scored on the tensor cores and selected in place
-    if (index_tc_fits(a.plan)) return launch_index_tc(a, s);
     const bool relu = (a.flags & CSA2_SCORE_RELU) != 0;
     const bool pool = a.plan.pool_blocks > 0 && !a.reindex;
     const void* fn = relu ? (pool ? (const void*)score_kernel<true, true> : (const void*)score_kernel<true, false>)

@@ -1,7 +1,10 @@
 """The workloads at full size, in the launch configuration bench.py times, checked against the
-oracle on every sequence (prefill: 72 query rows spread over the chunk, its first and last rows
-among them; multi-token decode: every row of every sequence): index sets and pools identical,
-attention within tolerance. The oracle runs in spawned host processes."""
+oracle: every sequence of the 1M-context Reindex and the Minimal workloads, 16 sequences spread over
+the batch of the 131,072-context Full workload, 72 query rows of the prefill chunk (its first and
+last rows among them) and every row of 16 sequences of the multi-token decode: index sets and pools
+identical, attention within tolerance. The oracle runs in spawned host processes (the sequences of
+the 131,072-context workloads and the 1M-position prefill cache take tens of seconds each to build
+on the host, which bounds how many of them fit in a test run)."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +16,7 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     ("full_b1_n4096", [0]),
-    ("full_b64_n131072", list(range(64))),
+    ("full_b64_n131072", list(range(0, 64, 4)) + [63]),
     ("reindex_b128_n1m", list(range(128))),
     ("minimal_b256_n262144", list(range(256))),
 ]
@@ -61,7 +64,7 @@ def test_prefill_workload_sampled_rows(orc):
     torch.cuda.synchronize()
     rows = sorted(set([0, 1, 2, 3, 2047, 4094, 4095] + list(range(5, 4096, 63))))
     assert len(rows) >= 64
-    groups = [rows[j::16] for j in range(16)]
+    groups = [rows[j::8] for j in range(8)]  # each process builds the 1M-position cache once
     r = oracle_steps(name, [0], rows=groups)[0]
     for i in rows:
         idx, ro, _ = r["rows"][i]
@@ -73,7 +76,7 @@ def test_prefill_workload_sampled_rows(orc):
 
 def test_draft_workload_sampled(orc):
     """Multi-token decode (5 draft tokens per sequence, 64 sequences at N = 131,072): the three calls
-    bench.py times; every row of every sequence against the oracle."""
+    bench.py times; every row of 17 sequences spread over the batch against the oracle."""
     import compressed_sparse_attention_append_b200 as csa
 
     step = G.build("draft_b64_n131072_tq5")
@@ -81,8 +84,9 @@ def test_draft_workload_sampled(orc):
     of = torch.empty(step.batch, wl.tq, 16, 128, dtype=torch.float32, device="cuda")
     step.run(out_f32=of)
     assert csa.csa2_get_device_status(step.ws) == 0
-    ref = oracle_steps("draft_b64_n131072_tq5", list(range(step.batch)))
-    for b in range(step.batch):
+    seqs = list(range(0, step.batch, 4)) + [step.batch - 1]
+    ref = oracle_steps("draft_b64_n131072_tq5", seqs)
+    for b in seqs:
         r = ref[b]
         for t in range(wl.tq):
             idx, ro, _ = r["rows"][t]
