@@ -203,6 +203,29 @@ struct RowCtr {            // per query row of the index step
     unsigned long long tau;// max over finished chunks of their local k-th key (lower bound)
 };
 
+// Several query rows per sequence on the tensor cores (index_mma.cu): block-scaled FP4 MMA scores
+// of 128-position key tiles against tiles of `nq` query rows; a sampled pass sets each row's
+// admission threshold, a full pass collects the positions above it, exact integer rescoring picks
+// the Top-k among them (index.cu).
+constexpr int kMmaTile = 128;     // key positions per tile
+constexpr int kMmaCap = 4096;     // candidates a row may rank (and positions it may rescore exactly)
+constexpr int kMmaTarget = 1536;  // candidates per row the sampled threshold aims at
+constexpr int64_t kMmaMinCtx = 8192;  // smaller contexts take the exact scan alone
+
+struct MmaPlan {
+    int on;            // 1: this plan runs the tensor-core filter (when the call allows it)
+    int nq;            // query columns per tile: 16 or 256
+    int nseq, nqt;     // sequences, query tiles per sequence
+    int nt;            // key tiles per sequence covering max_ctx
+    int st, ns;        // sampled key tiles: about every st-th tile, ns of them per sequence
+    int kc, nchunks;   // key tiles per filter work item, work items per (sequence, query tile)
+    int sc, nschunks;  // sampled tiles per sampling work item, items per (sequence, query tile)
+    int subcap;        // candidate slots of one row in one filter work item
+};
+
+// Key tile of sample s: one tile out of each run of st, at an offset that varies with s.
+__host__ __device__ inline int mma_sample_tile(int st, int s) { return s * st + (int)(((long long)s * 7) % st); }
+
 struct IndexPlan {
     int rows;          // batch * tq
     int k;
@@ -212,6 +235,7 @@ struct IndexPlan {
     int pool_blocks;   // 0 = no pool
     size_t cand_cap;   // candidate slots per row (decode rows: one key per position)
     int decode;        // 1: one query row per sequence, scored by score_kernel then select_kernel
+    MmaPlan mma;
 };
 
 struct AttendPlan {
@@ -245,6 +269,19 @@ struct WsLayout {
     size_t sel_key;    // u64[rows][2][kSelCand] (decode plans: candidate keys, then block maxima)
     size_t sel_pos;    // u64[rows][2][kSelCand] (element index << 32 | position, of each candidate)
     size_t att_part;   // f32[rows * splits * hq * kPartStride]
+    // tensor-core filter (several-row plans with mma.on); the first four are one zeroed range
+    size_t mma_zero, mma_zero_bytes;
+    size_t mma_smax;   // u32[nseq][16]: largest key scale byte of each 16-channel block
+    size_t mma_tend;   // u32[nseq * nqt]: key tiles visible to the rows of a query tile
+    size_t mma_fail_n; // u32: rows left to the exact scan
+    size_t mma_tm;     // u32[rows][ns]: orderable sampled tile maxima
+    size_t mma_cnt;    // u32[rows][nchunks]: candidates of a row found by each filter item
+    size_t mma_qc;     // u8[rows][128]: quantised query codes
+    size_t mma_qs;     // u8[rows][16]: their scales
+    size_t mma_row;    // float4[rows]: threshold estimate, error bound, admission threshold
+    size_t mma_cpos;   // i32[rows][nchunks][subcap]: candidate positions
+    size_t mma_cval;   // f32[rows][nchunks][subcap]: their approximate scores
+    size_t mma_fail;   // i32[rows]
     size_t total;
 };
 
@@ -278,6 +315,29 @@ inline IndexPlan make_index_plan(int rows, int tq, int k, int64_t max_scan, int 
     p.chunk_units = cu;
     p.chunks = (p.units_max + cu - 1) / cu;
     p.cand_cap = (size_t)p.chunks * (size_t)k;
+    if (max_scan >= kMmaMinCtx && k <= 1024 && pool_blocks == 0) {
+        MmaPlan& m = p.mma;
+        m.on = 1;
+        m.nq = tq <= 16 ? 16 : 256;
+        m.nseq = rows / tq;
+        m.nqt = (tq + m.nq - 1) / m.nq;
+        m.nt = (int)((max_scan + kMmaTile - 1) / kMmaTile);
+        int ns = m.nt / 16;
+        ns = ns < 64 ? 64 : (ns > 256 ? 256 : ns);
+        if (ns > m.nt) ns = m.nt;
+        m.st = (m.nt + ns - 1) / ns;
+        m.ns = (m.nt + m.st - 1) / m.st;
+        const long long pairs = (long long)m.nseq * m.nqt;
+        long long kc = (pairs * m.nt + 887) / 888;  // about six filter items per SM
+        m.kc = (int)(kc < 8 ? 8 : (kc > 64 ? 64 : kc));
+        m.nchunks = (m.nt + m.kc - 1) / m.kc;
+        // about three times the candidates a row expects from one item, plus headroom
+        const long long e = ((long long)kMmaTarget * m.kc + m.nt - 1) / m.nt;
+        m.subcap = (int)((3 * e + 16 + 15) / 16 * 16);
+        long long sc = (pairs * m.ns + 887) / 888;
+        m.sc = (int)(sc < 1 ? 1 : (sc > 16 ? 16 : sc));
+        m.nschunks = (m.ns + m.sc - 1) / m.sc;
+    }
     return p;
 }
 
@@ -320,6 +380,22 @@ inline WsLayout make_layout(const IndexPlan* ip, const AttendPlan* ap) {
     L.sel_pos = off; off = align256(off + drows * 2 * kSelCand * 8);
     size_t part = ap ? (size_t)ap->rows * (size_t)ap->splits * kHQ * kPartStride : 0;
     L.att_part = off; off = align256(off + 4 * part);
+    const bool mma = ip && ip->mma.on;
+    const size_t mrows = mma ? (size_t)rows_i : 0;
+    L.mma_zero = off;
+    L.mma_smax = off; off = align256(off + (mma ? 64 * (size_t)ip->mma.nseq : 0));
+    L.mma_tend = off; off = align256(off + (mma ? 4 * (size_t)ip->mma.nseq * ip->mma.nqt : 0));
+    L.mma_fail_n = off; off = align256(off + (mma ? 16 : 0));
+    L.mma_tm = off; off = align256(off + (mma ? 4 * mrows * ip->mma.ns : 0));
+    L.mma_zero_bytes = off - L.mma_zero;
+    const size_t nch = mma ? (size_t)ip->mma.nchunks : 0, sub = mma ? (size_t)ip->mma.subcap : 0;
+    L.mma_cnt = off; off = align256(off + 4 * mrows * nch);
+    L.mma_qc = off; off = align256(off + 128 * mrows);
+    L.mma_qs = off; off = align256(off + 16 * mrows);
+    L.mma_row = off; off = align256(off + 16 * mrows);
+    L.mma_cpos = off; off = align256(off + 4 * mrows * nch * sub);
+    L.mma_cval = off; off = align256(off + 4 * mrows * nch * sub);
+    L.mma_fail = off; off = align256(off + 4 * mrows);
     L.total = off;
     return L;
 }
@@ -357,9 +433,32 @@ struct IndexArgs {
     IndexPlan plan;
     unsigned char* ws;
     WsLayout L;
+    const int32_t* row_list;   // index_kernel: when set, only the rows listed (count *row_n) are scanned
+    const uint32_t* row_n;
 };
 cudaError_t launch_index(const IndexArgs& a, cudaStream_t s);         // index.cu: any tq
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t s);  // index_decode.cu: plan.decode
+// index_mma.cu: the tensor-core filter up to the candidate lists (the final selection is index.cu's)
+cudaError_t launch_index_mma(const IndexArgs& a, cudaStream_t s);
+
+// Last visible cache entry of query row `row` of an index call: -1 when none is visible yet, -2 for
+// a row whose token position is invalid (negative, or its entry at or past the capacity or max_ctx).
+__device__ __forceinline__ int64_t index_row_last(const IndexArgs& a, int row) {
+    const int64_t tok = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
+    if (tok < 0) return -2;
+    const int64_t q = (tok + 1) / a.ratio - 1;
+    if (q >= a.c.cap || q >= a.max_ctx) return -2;
+    return q;
+}
+
+// Orderable 32-bit image of a float (larger float <-> larger unsigned; 0 is below every image).
+__device__ __forceinline__ uint32_t f32_order(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float f32_unorder(uint32_t o) {
+    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
+}
 
 struct AttendArgs {
     csa2_cache c;

@@ -349,11 +349,9 @@ struct RowInfo {
 __device__ RowInfo row_info(const IndexArgs& a, int row) {
     RowInfo r;
     r.b = row / a.tq;
-    const int64_t tok = a.qpos ? a.qpos[row] : a.qpos_base + row % a.tq;
-    r.qpos = tok < 0 ? -1 : (tok + 1) / a.ratio - 1;  // the last visible entry
-    r.ok = true;
-    if (tok < 0 || r.qpos >= a.c.cap || r.qpos >= a.max_ctx) {
-        r.ok = false;
+    r.qpos = index_row_last(a, row);  // the last visible entry
+    r.ok = r.qpos >= -1;
+    if (!r.ok) {
         r.n_units = 0;
         return r;
     }
@@ -508,7 +506,8 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
     RowCtr* rctr = reinterpret_cast<RowCtr*>(ws + a.L.row_ctr);
     unsigned long long* cand_key = reinterpret_cast<unsigned long long*>(ws + a.L.cand_key);
     int* cand_pos = reinterpret_cast<int*>(ws + a.L.cand_pos);
-    const int rows = a.plan.rows;
+    // rows handed over by the tensor-core filter, or every row
+    const int rows = a.row_list ? (int)*(volatile const uint32_t*)a.row_n : a.plan.rows;
     const int total = rows * a.plan.chunks;
     unsigned char* wst = staging + warp * kStages * kStepBytes;
 
@@ -519,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
         __syncthreads();
         if (item >= total) break;
         const int chunk = item / rows;
-        const int row = item % rows;
+        const int row = a.row_list ? a.row_list[item % rows] : item % rows;
         const RowInfo R = row_info(a, row);
         RowCtr* rc = rctr + row;
         if (!R.ok && chunk == 0 && tid == 0) set_status(status, CSA2_DEV_BAD_POS);
@@ -654,17 +653,248 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
     }
 }
 
+// ---- final selection of the tensor-core filter (index_mma.cu): one CTA per row ----------------------
+// The k-th largest of n orderable values in shared memory (n >= k >= 1), built bit by bit: the
+// largest x with #{v >= x} >= k.
+__device__ uint32_t kth_largest_u32(const uint32_t* v, int n, int k, unsigned int* red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t x = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t y = x | (1u << bit);
+        unsigned int c = 0;
+        for (int i = tid; i < n; i += kThreads) c += v[i] >= y;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (lane == 0) red[warp] = c;
+        __syncthreads();
+        unsigned int tot = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) tot += red[w];
+        __syncthreads();
+        if (tot >= (unsigned)k) x = y;
+    }
+    return x;
+}
+
+// Shared memory: candidate images u32[kMmaCap] | candidate positions i32[kMmaCap] | rescored keys
+// u64[kMmaCap] | their positions i32[kMmaCap] | Top-k keys u64[k] | Top-k positions i32[k].
+size_t final_smem_bytes(int k) { return (size_t)20 * kMmaCap + (size_t)12 * k; }
+
+// Per row: gathers the candidates of the filter's work items, checks the conditions under which
+// they contain the exact Top-k, rescores {S^ >= A - 2 eps} exactly and ranks it (a row seeing at
+// most kMmaCap positions rescores all of them); a row failing a condition is listed for the exact
+// scan instead.
+__global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ Scal S;
+    __shared__ unsigned int hist[256];
+    __shared__ int kf_lut[256];
+    __shared__ unsigned int nabove, nsel, bad, ntot;
+    __shared__ unsigned int coff[256];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = blockIdx.x, K = a.plan.k;
+    const MmaPlan& P = a.plan.mma;
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(smem);
+    int* cposs = reinterpret_cast<int*>(ckey + kMmaCap);
+    unsigned long long* rkey = reinterpret_cast<unsigned long long*>(cposs + kMmaCap);
+    int* rpos = reinterpret_cast<int*>(rkey + kMmaCap);
+    unsigned long long* okey = reinterpret_cast<unsigned long long*>(rpos + kMmaCap);
+    int* opos = reinterpret_cast<int*>(okey + K);
+    uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + kHdrStatus);
+    int32_t* out = a.out_idx + (size_t)row * K;
+
+    const int64_t ql = index_row_last(a, row);
+    if (ql < -1 && tid == 0) set_status(status, CSA2_DEV_BAD_POS);
+    const int64_t n = ql + 1;
+    if (n <= K) {  // every visible position (none for an invalid row)
+        for (int i = tid; i < K; i += kThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    kf_lut[tid] = e4m3_fixed(tid);
+    const float4 rp = reinterpret_cast<const float4*>(a.ws + a.L.mma_row)[row];
+    const float tau = rp.x, eps = rp.y;
+    const bool whole = n <= kMmaCap;
+    if (tid == 0) { bad = 0; nsel = 0; nabove = 0; ntot = 0; }
+    __syncthreads();
+    bool ok = true;
+    if (whole) {
+        for (int i = tid; i < (int)n; i += kThreads) rpos[i] = i;
+        if (tid == 0) nsel = (unsigned)n;
+    } else {
+        // the row's lists, one per filter item over its visible key tiles
+        const int b = row / a.tq, j = (row % a.tq) / P.nq;
+        const int te = (int)reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_tend)[b * P.nqt + j];
+        const int nch = (te + P.kc - 1) / P.kc;
+        const uint32_t* cc = reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_cnt) + (size_t)row * P.nchunks;
+        if (warp == 0) {
+            unsigned int run = 0;
+            for (int c0 = 0; c0 < nch; c0 += 32) {
+                const int c = c0 + lane;
+                const unsigned int v = c < nch ? cc[c] : 0u;
+                if (v > (unsigned)P.subcap) atomicOr(&bad, 1u);
+                unsigned int incl = v;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += t;
+                }
+                if (c < nch && c < 256) coff[c] = run + incl - v;
+                run += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) { ntot = run; if (nch > 256) bad = 1; }
+        }
+        __syncthreads();
+        ok = bad == 0 && ntot <= (unsigned)kMmaCap;
+        if (ok) {
+            const float* cv = reinterpret_cast<const float*>(a.ws + a.L.mma_cval) + (size_t)row * P.nchunks * P.subcap;
+            const int* cp = reinterpret_cast<const int*>(a.ws + a.L.mma_cpos) + (size_t)row * P.nchunks * P.subcap;
+            const uint32_t otau = f32_order(tau);
+            unsigned int above = 0;
+            for (int f = tid; f < nch * P.subcap; f += kThreads) {
+                const int c = f / P.subcap, i = f - c * P.subcap;
+                if (i < (int)cc[c]) {
+                    const unsigned int o = coff[c] + i;
+                    ckey[o] = f32_order(cv[f]);
+                    cposs[o] = cp[f];
+                    above += ckey[o] >= otau;
+                }
+            }
+            above = __reduce_add_sync(0xffffffffu, above);
+            if (lane == 0 && above) atomicAdd(&nabove, above);
+            __syncthreads();
+            ok = nabove >= (unsigned)K;  // at least k positions above the estimate
+        }
+        if (ok) {
+            const int cnt = (int)ntot;
+            const float A = f32_unorder(kth_largest_u32(ckey, cnt, K, hist));
+            const uint32_t olo = f32_order(__double2float_rd((double)A - 2.0 * (double)eps));
+            for (int base = 0; base < cnt; base += kThreads) {
+                const int i = base + tid;
+                const bool v = i < cnt && ckey[i] >= olo;
+                const unsigned int bal = __ballot_sync(0xffffffffu, v);
+                unsigned int wb = 0;
+                if (lane == 0 && bal) wb = atomicAdd(&nsel, (unsigned)__popc(bal));
+                wb = __shfl_sync(0xffffffffu, wb, 0);
+                if (v) {
+                    const unsigned int o = wb + __popc(bal & ((1u << lane) - 1u));
+                    rkey[o] = ckey[i];
+                    rpos[o] = cposs[i];
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (ok) {
+        // the query exactly as the tensor cores saw it, as the integer words of score_step
+        const uint8_t* qc = a.ws + a.L.mma_qc + (size_t)row * kIKBytes;
+        if (tid < 128) S.qcode[tid] = qc[tid];
+        if (tid < 16) S.qf[tid] = kf_lut[a.ws[a.L.mma_qs + (size_t)row * kIKScales + tid]];
+        __syncthreads();
+        if (tid < 128) {
+            const int cs = tid >> 4, wi = (tid >> 2) & 3, kind = tid & 3;
+            const uint32_t cw = *reinterpret_cast<const uint32_t*>(&S.qcode[16 * cs + 4 * wi]);
+            uint32_t r = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t vq = e2m1_int2((cw >> (4 * j + ((kind & 1) ? 16 : 0))) & 15);
+                if (kind & 2) vq = (0u - vq) & 0xFF;
+                r |= vq << (8 * j);
+            }
+            S.qv[tid] = r;
+        }
+        __syncthreads();
+        // exact scores: 8 threads per position, each 32 channels (two scale blocks)
+        const int sub = lane & 7, grp = tid >> 3;
+        uint32_t qv[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 q4 = *reinterpret_cast<const uint4*>(&S.qv[16 * sub + 4 * i]);
+            qv[4 * i + 0] = q4.x; qv[4 * i + 1] = q4.y; qv[4 * i + 2] = q4.z; qv[4 * i + 3] = q4.w;
+        }
+        const int qf0 = S.qf[2 * sub], qf1 = S.qf[2 * sub + 1];
+        const int nr = (int)nsel;
+        const int b = row / a.tq;
+        const uint8_t* kbase = a.c.ik_data + (size_t)b * a.c.cap * kIKBytes;
+        const uint8_t* sbase = a.c.ik_scale + (size_t)b * a.c.cap * kIKScales;
+        constexpr int kG = kThreads / 8;  // positions per round and unrolled group
+        for (int base = 0; base < nr; base += 4 * kG) {
+            uint4 w[4];
+            uint32_t sc[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const int i = base + h * kG + grp;
+                w[h] = make_uint4(0, 0, 0, 0);
+                sc[h] = 0;
+                if (i < nr) {
+                    const size_t p = (size_t)rpos[i];
+                    w[h] = __ldg(reinterpret_cast<const uint4*>(kbase + p * kIKBytes + 16 * sub));
+                    sc[h] = __ldg(reinterpret_cast<const uint16_t*>(sbase + p * kIKScales + 2 * sub));
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const int i = base + h * kG + grp;
+                int d0 = dot8(w[h].x, qv[0], qv[1], qv[2], qv[3], 0);
+                d0 = dot8(w[h].y, qv[4], qv[5], qv[6], qv[7], d0);
+                int d1 = dot8(w[h].z, qv[8], qv[9], qv[10], qv[11], 0);
+                d1 = dot8(w[h].w, qv[12], qv[13], qv[14], qv[15], d1);
+                long long v = (long long)(d0 * kf_lut[sc[h] & 0xFF]) * qf0 + (long long)(d1 * kf_lut[sc[h] >> 8]) * qf1;
+                v += shfl_xor_s64(v, 1);
+                v += shfl_xor_s64(v, 2);
+                v += shfl_xor_s64(v, 4);
+                if (sub == 0 && i < nr) {
+                    if (!whole) {  // the error bound held for this position
+                        const double shat = (double)f32_unorder((uint32_t)rkey[i]);
+                        if (fabs(shat - (double)v * 0x1p-20) > (double)eps) atomicOr(&bad, 1u);
+                    }
+                    rkey[i] = (unsigned long long)v ^ 0x8000000000000000ull;
+                }
+            }
+        }
+        __syncthreads();
+        ok = bad == 0;
+    }
+    if (!ok) {  // the exact scan takes this row
+        if (tid == 0) {
+            const unsigned int f = atomicAdd(reinterpret_cast<uint32_t*>(a.ws + a.L.mma_fail_n), 1u);
+            reinterpret_cast<int32_t*>(a.ws + a.L.mma_fail)[f] = row;
+        }
+        return;
+    }
+    if (tid == 0) S.thr = 0;
+    __syncthreads();
+    cta_select(rkey, rpos, (int)nsel, nullptr, nullptr, 0, K, okey, opos, hist, S);
+    int* buf = reinterpret_cast<int*>(rkey);  // kMmaCap ints >= the next power of two of K
+    for (int i = tid; i < K; i += kThreads) buf[i] = opos[i];
+    __syncthreads();
+    sort_ascending(buf, K);
+    for (int i = tid; i < K; i += kThreads) out[i] = buf[i];
+}
+
 size_t smem_bytes(const IndexPlan& p) {
     return (size_t)kStagingBytes + (size_t)12 * (2 * p.k + kNewCap);
 }
 
 }  // namespace
 
-cudaError_t launch_index(const IndexArgs& a, cudaStream_t s) {
+cudaError_t launch_index(const IndexArgs& a0, cudaStream_t s) {
     // rows of one query per sequence (Full with a pool, Reindex) take index_decode.cu
-    if (a.reindex || a.plan.pool_blocks > 0) return cudaErrorInvalidValue;
+    if (a0.reindex || a0.plan.pool_blocks > 0) return cudaErrorInvalidValue;
+    const bool relu = (a0.flags & CSA2_SCORE_RELU) != 0;
+    IndexArgs a = a0;
+    if (a.plan.mma.on && !relu && a.ratio == 1) {
+        // tensor-core filter and exact final selection; the rows it hands back take the exact scan
+        cudaError_t e = launch_index_mma(a, s);
+        if (e != cudaSuccess) return e;
+        const size_t fs = final_smem_bytes(a.plan.k);
+        e = cudaFuncSetAttribute(mma_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fs);
+        if (e != cudaSuccess) return e;
+        mma_final_kernel<<<(unsigned)a.plan.rows, kThreads, fs, s>>>(a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        a.row_list = reinterpret_cast<const int32_t*>(a.ws + a.L.mma_fail);
+        a.row_n = reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_fail_n);
+    }
     const size_t smem = smem_bytes(a.plan);
-    const bool relu = (a.flags & CSA2_SCORE_RELU) != 0;
     const void* fn = relu ? (const void*)index_kernel<true> : (const void*)index_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -674,7 +904,7 @@ cudaError_t launch_index(const IndexArgs& a, cudaStream_t s) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
-    const long long items = (long long)a.plan.rows * a.plan.chunks;
+    const long long items = (long long)a.plan.rows * a.plan.chunks;  // at most (row list: fewer)
     long long grid = (long long)sms * per_sm;
     if (grid > items) grid = items;
     if (grid < 1) grid = 1;

@@ -80,6 +80,66 @@ def test_full_mode_multi_row_queries(orc, tq, ratio):
             assert np.array_equal(out[b * tq + t].cpu().numpy(), ref), (b, t)
 
 
+@pytest.mark.parametrize("B,tq,n,k", [(1, 300, 20000, 512), (3, 5, 20000, 512), (2, 40, 9000, 256)])
+def test_full_mode_multi_row_tensor_core(orc, B, tq, n, k):
+    """Several rows per sequence at a context that takes the tensor-core filter (approximate MMA
+    scores, exact rescoring of the survivors): index sets identical to the oracle's. The rows mix
+    the cases of that path: the usual sampled threshold, a row whose visible prefix fits the
+    candidate list (every position admitted), a row seeing fewer than k positions, and an all-zero
+    query (every score equal: the candidate list overflows and the exact scan takes the row)."""
+    seed = 17 + tq
+    shape, cache, swa_cap = _setup(B, n, seed)
+    rng = np.random.default_rng(seed)
+    qpos = [[n - 1 - int(rng.integers(0, n // 4)) for _ in range(tq)] for _ in range(B)]
+    qpos[0][0] = n - 1
+    if tq > 2:
+        qpos[0][1] = 3000          # visible prefix within the candidate list
+        qpos[0][2] = k // 2        # fewer than k visible positions
+    qp = torch.tensor(qpos, dtype=torch.int64, device=DEV).reshape(-1)
+    rows_b = torch.arange(B).repeat_interleave(tq)
+    iq = query_values(seed, "iq", rows_b.to(DEV), qp, 256, DEV).contiguous()
+    zero_row = B * tq - 1
+    iq[zero_row] = 0
+    out = torch.full((B * tq, k), -7, dtype=torch.int32, device=DEV)
+    ws = csa.Workspace(shape, B, tq, k, n)
+    for rep in range(2):
+        csa.csa2_index_topk_full(shape, cache, B, tq, qp, iq, k, out, max_ctx=n, ws=ws)
+        assert csa.csa2_get_device_status(ws) == 0
+        for b in range(B):
+            oc = oracle_seq(seed, b, n, n, swa_cap)
+            for t in range(tq):
+                r = b * tq + t
+                qb = iq[r].cpu() if r == zero_row else query_values(seed, "iq", [b], [qpos[b][t]], 256, "cpu")[0]
+                ref = oc.index_topk_full(qpos[b][t], bf16_np(qb), k=k)
+                assert np.array_equal(out[r].cpu().numpy(), ref), (rep, b, t)
+
+
+def test_prefill_chunk_tensor_core_blind_sample(orc):
+    """A prefill chunk over a context where every 5th key is 8x larger: the sampled tile maxima see
+    mostly those keys; the selection must still be exact (through the filter, or the exact scan for
+    rows whose threshold admitted fewer than k keys)."""
+    n, t, k = 12000, 64, 512
+    p = torch.arange(n)
+    ik = values(8, "ik", [0], p, 256, "cpu")[0].float()
+    ik[p % 5 == 0] *= 8.0
+    ik = ik.to(torch.bfloat16)
+    shape = csa.make_shape()
+    cache = csa.Cache(1, n, 1 << 14)
+    ws = csa.Workspace(shape, 1, t, k, n)
+    pos = torch.zeros(1, dtype=torch.int64, device=DEV)
+    csa.csa2_quantize_append(shape, cache, 1, n, pos, None, ik[None].to(DEV).contiguous(), None, ws=ws)
+    qpos = torch.arange(n - t, n, dtype=torch.int64)
+    iq = query_values(8, "iq", torch.zeros(t, dtype=torch.int64), qpos, 256, "cpu").contiguous()
+    out = torch.full((t, k), -7, dtype=torch.int32, device=DEV)
+    csa.csa2_index_topk_full(shape, cache, 1, t, qpos.to(DEV), iq.to(DEV), k, out, max_ctx=n, ws=ws)
+    assert csa.csa2_get_device_status(ws) == 0
+    oc = oracle.SeqCache(n, 1 << 14)
+    oc.append(0, idx_k=bf16_np(ik))
+    for r in range(0, t, 7):
+        ref = oc.index_topk_full(int(qpos[r]), bf16_np(iq[r]), k=k)
+        assert np.array_equal(out[r].cpu().numpy(), ref), r
+
+
 def test_full_mode_long_pool(orc):
     """More pool blocks than fit on chip (17,500 blocks of 8): the pool ranking reads from memory."""
     B, n, k, P = 1, 140000, 64, 256
