@@ -52,7 +52,8 @@ def algorithmic_bytes(wl):
         index = wl.context * 144 / wl.tq + iq + idx
         append = 3 * 256 * 2 + 144 * 2 + 256
     else:
-        index = wl.context * 144 + iq + idx  # per query row (upper bound: the last row sees all)
+        # prefill chunk: the chunk's rows share one pass over the visible indexer keys
+        index = wl.context * 144 / wl.tq + iq + idx
         append = 3 * 256 * 2 + 144 * 2 + 256
     return {"append": append, "index": index, "attend": attend}
 
@@ -60,14 +61,22 @@ def algorithmic_bytes(wl):
 L2_BYTES = 126 * 1024 * 1024
 
 
+def tensor_core_index(wl):
+    """Several rows per sequence at a context of 8,192 or more (and k <= 1024) take the tensor-core
+    filter of index_mma.cu."""
+    return wl.mode in ("prefill", "draft") and wl.context >= 8192 and wl.k <= 1024
+
+
 def kernels_per_step(wl):
-    """Kernels one step launches: append 1; index: 3 for decode rows (zero + score + select), 1 for
-    several rows per sequence (the multi-row kernel); attention 1."""
+    """Kernels one step launches: append 1; index: 3 for decode rows (zero + score + select); for
+    several rows per sequence 6 on the tensor-core path (prep, sampled pass, threshold, filter, final
+    selection, and the exact scan, which returns at once when no row was handed back), else 1;
+    attention 1."""
     if wl.mode == "minimal":
         return 2
     if wl.mode in ("full", "reindex"):
         return 5
-    return 3
+    return 8 if tensor_core_index(wl) else 3
 
 
 def measured_peaks():
@@ -77,6 +86,18 @@ def measured_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def fp4_tensor_peak():
+    """Dense FP4 tensor TFLOP/s: the measured bf16 GEMM burst figure times the nominal FP4 : bf16
+    ratio (9 : 2.25 PFLOP/s dense = 4)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return 4.0 * float(d["bf16_tflops"]), "measured bf16 burst x 4"
+    return 4.0 * 1590.0, "fallback bf16 1.59 PFLOP/s x 4"
 
 
 def kernel_source_hash(name):
@@ -415,7 +436,7 @@ def run_gpu(args):
         if world > 1:
             dist.barrier()
 
-    kern = ("append", "index", "attend") if wl.mode != "prefill" else ("prefill",)
+    kern = ("append", "index", "attend")
     ev = {k: [] for k in kern}
     # a step that reads less than the L2 holds is timed step by step with L2 flushed in between
     step_read = sum(algorithmic_bytes(wl).values()) * B * wl.tq
@@ -446,12 +467,7 @@ def run_gpu(args):
                 scrub.zero_()  # writes twice the L2: the step reads its inputs from HBM
                 e0 = torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
-            if wl.mode == "prefill":
-                hook("prefill", 0)
-                step.run()
-                hook("prefill", 1)
-            else:
-                step.run_parts(hook)
+            step.run_parts(hook)
             if flush:
                 e1 = torch.cuda.Event(enable_timing=True)
                 e1.record(stream)
@@ -480,20 +496,31 @@ def run_gpu(args):
     ab = algorithmic_bytes(wl)
     # every kernel of the step against the HBM roofline (algorithmic bytes / its event time)
     per_kernel = {}
-    if wl.mode != "prefill":
-        for k, t_ms in kms.items():
-            if t_ms > 0 and ab.get(k):
-                nbytes = ab[k] * B * wl.tq
-                per_kernel[k] = {"algorithmic_bytes_per_launch": int(round(nbytes)), "ms_per_launch": round(t_ms, 5),
-                                 "achieved_gbs": round(nbytes / (t_ms / 1e3) / 1e9, 1),
-                                 "frac": round(nbytes / (t_ms / 1e3) / 1e9 / peak, 4)}
-    dom = "index" if wl.mode in ("full", "reindex", "draft") else ("attend" if wl.mode == "minimal" else "prefill")
-    if dom == "prefill":
-        dom_bytes = (ab["index"] + ab["attend"]) * wl.tq
-        dom_file, dom_kernels = "index.cu", "index_kernel + attend_kernel"
+    tpeak, tpeak_kind = fp4_tensor_peak()
+    # the prefill chunk's index step is a contraction: rows x visible positions x 256 channels
+    p0 = wl.context - wl.tq
+    macs = 256.0 * (wl.tq * p0 + wl.tq * (wl.tq + 1) / 2.0) * B
+    for k, t_ms in kms.items():
+        if t_ms <= 0:
+            continue
+        if wl.mode == "prefill" and k == "index":
+            tf = 2.0 * macs / (t_ms / 1e3) / 1e12
+            per_kernel[k] = {"bound": "tensor", "flops_per_launch": 2.0 * macs, "ms_per_launch": round(t_ms, 5),
+                             "achieved_tflops": round(tf, 1), "frac": round(tf / tpeak, 4)}
+        elif ab.get(k):
+            nbytes = ab[k] * B * wl.tq
+            per_kernel[k] = {"algorithmic_bytes_per_launch": int(round(nbytes)), "ms_per_launch": round(t_ms, 5),
+                             "achieved_gbs": round(nbytes / (t_ms / 1e3) / 1e9, 1),
+                             "frac": round(nbytes / (t_ms / 1e3) / 1e9 / peak, 4)}
+    dom = "attend" if wl.mode == "minimal" else "index"
+    mma_kernels = ("mma_prep_kernel + mma_score_kernel (sampled pass) + mma_tau_kernel + mma_score_kernel "
+                   "(tensor-core filter) + mma_final_kernel + index_kernel (rows handed back)")
+    if wl.mode == "prefill":
+        dom_bytes = None
+        dom_file, dom_kernels = "index_mma.cu", mma_kernels
     elif wl.mode == "draft":
         dom_bytes = int(round(ab[dom] * B * wl.tq))
-        dom_file, dom_kernels = "index.cu", "index_kernel"
+        dom_file, dom_kernels = ("index_mma.cu", mma_kernels) if tensor_core_index(wl) else ("index.cu", "index_kernel")
     else:
         dom_bytes = ab[dom] * B
         # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
@@ -502,18 +529,14 @@ def run_gpu(args):
         else:
             dom_file, dom_kernels = "attend.cu", "attend_kernel"
     dur_s = kms[dom] / 1e3
-    if dom == "prefill":
-        # the prefill chunk scores every visible (row, position) pair with dp4a on the CUDA cores:
-        # bound by integer issue. Useful multiply-adds per chunk: rows x visible positions x 256
-        # channels; peak = 148 SMs x 64 dp4a lanes per clock x 4 multiply-adds x 1.965 GHz.
-        visible = wl.context - wl.tq + (wl.tq + 1) / 2.0
-        macs = wl.tq * visible * 256
-        achieved = macs / dur_s / 1e12
-        alu_peak = 148 * 64 * 4 * 1.965e9 / 1e12
-        roof = {"kernel": dom, "kernels": dom_kernels, "bound": "alu", "achieved": round(achieved, 2),
-                "peak": round(alu_peak, 1), "unit": "TMAC/s", "frac": round(achieved / alu_peak, 4),
-                "peak_kind": "derived (dp4a issue rate x clock)", "traffic": None,
-                "macs_per_launch": macs, "ms_per_launch": round(kms[dom], 5)}
+    if wl.mode == "prefill":
+        # block-scaled FP4 MMA of every visible (row, position) pair of the chunk: 2 x rows x visible
+        # positions x 256 channels of FP4 tensor work per index step, against the dense FP4 peak
+        achieved = 2.0 * macs / dur_s / 1e12
+        roof = {"kernel": dom, "kernels": dom_kernels, "bound": "tensor", "achieved": round(achieved, 1),
+                "peak": round(tpeak, 1), "unit": "TFLOP/s", "frac": round(achieved / tpeak, 4),
+                "peak_kind": tpeak_kind, "traffic": None, "flops_per_launch": 2.0 * macs,
+                "ms_per_launch": round(kms[dom], 5)}
     else:
         achieved = dom_bytes / dur_s / 1e9
         roof = {"kernel": dom, "kernels": dom_kernels, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,

@@ -654,36 +654,64 @@ __global__ void __launch_bounds__(kThreads, 2) index_kernel(IndexArgs a) {
 }
 
 // ---- final selection of the tensor-core filter (index_mma.cu): one CTA per row ----------------------
-// The k-th largest of n orderable values in shared memory (n >= k >= 1), built bit by bit: the
-// largest x with #{v >= x} >= k.
-__device__ uint32_t kth_largest_u32(const uint32_t* v, int n, int k, unsigned int* red) {
+// A lower bound of the k-th largest of n orderable values in shared memory (n >= k >= 1): that value
+// with its low 8 bits cleared (three 8-bit radix passes), so at least k values are >= the result.
+__device__ uint32_t kth_lower_bound(const uint32_t* v, int n, int k, unsigned int* hist, Scal& S) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t x = 0;
-    for (int bit = 31; bit >= 0; --bit) {
-        const uint32_t y = x | (1u << bit);
-        unsigned int c = 0;
-        for (int i = tid; i < n; i += kThreads) c += v[i] >= y;
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (lane == 0) red[warp] = c;
+    uint32_t prefix = 0, mask = 0;
+    int kr = k;
+    for (int shift = 24; shift >= 8; shift -= 8) {
+        hist[tid] = 0;
         __syncthreads();
-        unsigned int tot = 0;
+        for (int i = tid; i < n; i += kThreads)
+            if ((v[i] & mask) == prefix) atomicAdd(&hist[(v[i] >> shift) & 255u], 1u);
+        __syncthreads();
+        if (warp == 0) {
+            // lane L owns bins 255-8L ... 248-8L (descending)
+            unsigned int c[8], sum = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) tot += red[w];
+            for (int j = 0; j < 8; ++j) { c[j] = hist[255 - 8 * lane - j]; sum += c[j]; }
+            unsigned int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const unsigned int excl = incl - sum;
+            if (excl < (unsigned)kr && incl >= (unsigned)kr) {
+                unsigned int run = excl;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (run + c[j] >= (unsigned)kr) {
+                        S.digit = 255 - 8 * lane - j;
+                        S.above = (int)run;
+                        break;
+                    }
+                    run += c[j];
+                }
+            }
+        }
         __syncthreads();
-        if (tot >= (unsigned)k) x = y;
+        kr -= S.above;
+        prefix |= (uint32_t)S.digit << shift;
+        mask |= 255u << shift;
+        __syncthreads();
     }
-    return x;
+    return prefix;
 }
 
-// Shared memory: candidate images u32[kMmaCap] | candidate positions i32[kMmaCap] | rescored keys
-// u64[kMmaCap] | their positions i32[kMmaCap] | Top-k keys u64[k] | Top-k positions i32[k].
-size_t final_smem_bytes(int k) { return (size_t)20 * kMmaCap + (size_t)12 * k; }
+// Shared memory (64 KB, three CTAs per SM): A0 = u32[kMmaCap], A1 = i32[kMmaCap], B = u64[kMmaCap].
+// Filtered rows: candidate images in A0 and positions in A1, then the rescored set's positions in A0
+// and keys in B, the Top-k (u64[k] keys, i32[k] positions) in A1. Rows rescored whole: positions in
+// A1, keys in B, the Top-k in A0.
+size_t final_smem_bytes(int) { return (size_t)16 * kMmaCap; }
 
 // Per row: gathers the candidates of the filter's work items, checks the conditions under which
-// they contain the exact Top-k, rescores {S^ >= A - 2 eps} exactly and ranks it (a row seeing at
+// they contain the exact Top-k, rescores {S^ >= A - 2 eps} exactly (A: a lower bound of the k-th
+// largest S^ among the candidates, so at least k of them are >= A) and ranks it (a row seeing at
 // most kMmaCap positions rescores all of them); a row failing a condition is listed for the exact
 // scan instead.
-__global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) mma_final_kernel(IndexArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ Scal S;
     __shared__ unsigned int hist[256];
@@ -693,12 +721,12 @@ __global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = blockIdx.x, K = a.plan.k;
     const MmaPlan& P = a.plan.mma;
-    uint32_t* ckey = reinterpret_cast<uint32_t*>(smem);
-    int* cposs = reinterpret_cast<int*>(ckey + kMmaCap);
-    unsigned long long* rkey = reinterpret_cast<unsigned long long*>(cposs + kMmaCap);
-    int* rpos = reinterpret_cast<int*>(rkey + kMmaCap);
-    unsigned long long* okey = reinterpret_cast<unsigned long long*>(rpos + kMmaCap);
-    int* opos = reinterpret_cast<int*>(okey + K);
+    static_assert(kMmaCap % kThreads == 0 && kMmaCap / kThreads <= 16, "two-phase compaction registers");
+    unsigned char* A0 = smem;
+    unsigned char* A1 = smem + 4 * kMmaCap;
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(A0);
+    int* cposs = reinterpret_cast<int*>(A1);
+    unsigned long long* rkey = reinterpret_cast<unsigned long long*>(smem + 8 * kMmaCap);
     uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + kHdrStatus);
     int32_t* out = a.out_idx + (size_t)row * K;
 
@@ -713,6 +741,9 @@ __global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
     const float4 rp = reinterpret_cast<const float4*>(a.ws + a.L.mma_row)[row];
     const float tau = rp.x, eps = rp.y;
     const bool whole = n <= kMmaCap;
+    int* rpos = reinterpret_cast<int*>(whole ? A1 : A0);
+    unsigned long long* okey = reinterpret_cast<unsigned long long*>(whole ? A0 : A1);
+    int* opos = reinterpret_cast<int*>(okey + K);
     if (tid == 0) { bad = 0; nsel = 0; nabove = 0; ntot = 0; }
     __syncthreads();
     bool ok = true;
@@ -749,13 +780,14 @@ __global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
             const int* cp = reinterpret_cast<const int*>(a.ws + a.L.mma_cpos) + (size_t)row * P.nchunks * P.subcap;
             const uint32_t otau = f32_order(tau);
             unsigned int above = 0;
-            for (int f = tid; f < nch * P.subcap; f += kThreads) {
-                const int c = f / P.subcap, i = f - c * P.subcap;
-                if (i < (int)cc[c]) {
-                    const unsigned int o = coff[c] + i;
-                    ckey[o] = f32_order(cv[f]);
-                    cposs[o] = cp[f];
-                    above += ckey[o] >= otau;
+            for (int c = warp; c < nch; c += kWarps) {  // one warp per list
+                const int m = (int)cc[c];
+                const size_t src = (size_t)c * P.subcap;
+                for (int i = lane; i < m; i += 32) {
+                    const uint32_t o = f32_order(cv[src + i]);
+                    ckey[coff[c] + i] = o;
+                    cposs[coff[c] + i] = cp[src + i];
+                    above += o >= otau;
                 }
             }
             above = __reduce_add_sync(0xffffffffu, above);
@@ -765,21 +797,43 @@ __global__ void __launch_bounds__(kThreads, 2) mma_final_kernel(IndexArgs a) {
         }
         if (ok) {
             const int cnt = (int)ntot;
-            const float A = f32_unorder(kth_largest_u32(ckey, cnt, K, hist));
+            const float A = f32_unorder(kth_lower_bound(ckey, cnt, K, hist, S));
             const uint32_t olo = f32_order(__double2float_rd((double)A - 2.0 * (double)eps));
-            for (int base = 0; base < cnt; base += kThreads) {
-                const int i = base + tid;
-                const bool v = i < cnt && ckey[i] >= olo;
-                const unsigned int bal = __ballot_sync(0xffffffffu, v);
-                unsigned int wb = 0;
-                if (lane == 0 && bal) wb = atomicAdd(&nsel, (unsigned)__popc(bal));
-                wb = __shfl_sync(0xffffffffu, wb, 0);
-                if (v) {
-                    const unsigned int o = wb + __popc(bal & ((1u << lane) - 1u));
-                    rkey[o] = ckey[i];
-                    rpos[o] = cposs[i];
+            // two-phase compaction of {S^ >= A - 2 eps} (the positions then overwrite A0): every
+            // element is read into registers before any is written, output in candidate order
+            constexpr int kPer = kMmaCap / kThreads;
+            uint32_t kr[kPer];
+            int pr[kPer];
+            unsigned int sel = 0, mine = 0;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = j * kThreads + tid;
+                kr[j] = 0;
+                pr[j] = 0;
+                if (i < cnt) {
+                    kr[j] = ckey[i];
+                    pr[j] = cposs[i];
+                    if (kr[j] >= olo) { sel |= 1u << j; ++mine; }
                 }
             }
+            unsigned int incl = mine;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            if (lane == 31) coff[warp] = incl;
+            __syncthreads();
+            unsigned int base = incl - mine;
+            for (int w = 0; w < warp; ++w) base += coff[w];
+            if (tid == kThreads - 1) nsel = base + mine;
+#pragma unroll
+            for (int j = 0; j < kPer; ++j)
+                if (sel & (1u << j)) {
+                    rkey[base] = kr[j];
+                    rpos[base] = pr[j];
+                    ++base;
+                }
         }
     }
     __syncthreads();

@@ -28,12 +28,14 @@
 // sum of |terms| (576 = 16 channels x 6 x 6), far above the rounding of fp32 accumulation of 256
 // terms (about 2^-23 of that sum, as measured).
 //
-// Kernel roles (320 threads, one CTA per SM with 256 query columns, two with 16): warp 0 issues the
-// TMA copies of key tiles (codes through a 128-byte-swizzled tensor map, scales by a bulk copy)
+// Kernel roles (one CTA of 14 warps per SM with 256 query columns, two of 10 with 16): warp 0 issues
+// the TMA copies of key tiles (codes through a 128-byte-swizzled tensor map, scales by a bulk copy)
 // into a 4-stage ring; warp 1 turns the scales into tensor-core scale-factor matrices
 // (tcgen05.cp, replicated over the four lane quadrants) and issues the MMAs into tensor-memory
-// accumulator slots; warps 2-9 read the accumulators (tcgen05.ld, two warps per lane quadrant,
-// alternating slots) and either admit candidates or reduce tile maxima. Every wait is bounded: one
+// accumulator slots; the other warps, in sets of four (one per lane quadrant) taking the slots in
+// turn, read the accumulators (tcgen05.ld) and either admit candidates or reduce tile maxima. A
+// candidate goes to the list its row keeps for this work item, counted in shared memory: each
+// (row, item) list has one writer CTA, so no global atomics are needed. Every wait is bounded: one
 // that runs out sets CSA2_DEV_TIMEOUT, and the CTA winds down (the producer waits for its copies in
 // flight and the MMA warp for its MMAs, with the same bound) and frees its tensor memory.
 #include <mutex>
@@ -52,8 +54,6 @@ constexpr int kSt = 4;                         // key tile stages
 constexpr int kCodeB = kTP * kIKBytes;         // 16384
 constexpr int kScB = kTP * kIKScales;          // 2048
 constexpr int kStageB = kCodeB + 2 * kScB;     // codes | raw scales | scale-factor matrices
-constexpr int kEpi = 8;                        // accumulator-reading warps
-constexpr int kThr = 32 * (2 + kEpi);
 constexpr uint64_t kWaitNs = 200000000ull;     // bound of one pipeline wait
 constexpr float kEpsRel = 1.0f / 16384.0f;     // 2^-14
 
@@ -62,15 +62,22 @@ struct Cfg {
     static constexpr int W = NQ > 128 ? 128 : NQ;   // MMA N
     static constexpr int H = NQ / W;                // MMAs per K step
     static constexpr int NSLOT = NQ > 128 ? 3 : 8;  // accumulator slots of W columns
+    static constexpr int SETS = NQ > 128 ? 3 : 2;   // sets of four accumulator-reading warps (one per
+                                                    // lane quadrant); set u % SETS reads slot use u
+    static constexpr int EPI = 4 * SETS;
+    static constexpr int THREADS = 32 * (2 + EPI);
     static constexpr int SFA = NSLOT * W;           // key scale factors: 16 columns per stage
     static constexpr int SFB = SFA + 16 * kSt;      // query scale factors: 16 columns per half
     static constexpr int COLS = SFB + 16 * H <= 256 ? 256 : 512;
     static constexpr int BQ = NQ * kIKBytes;        // query tile bytes
     static constexpr int CH = W < 32 ? W : 32;      // accumulator columns per tcgen05.ld
-    static constexpr size_t SMEM = 1024 + BQ + (size_t)kSt * kStageB + (size_t)NQ * 12 + 8 * (2 * kSt + 2 * NSLOT + 2);
+    static constexpr int HS = CH + 4;               // floats per lane of a warp's hit staging rows
+    static constexpr size_t SMEM = 1024 + BQ + (size_t)kSt * kStageB + (size_t)NQ * 12 +
+                                   (size_t)EPI * 32 * HS * 4 + 8 * (2 * kSt + 2 * NSLOT + 2);
 };
 
-__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpi) : "memory"); }
+template <int EPI>
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, %0;" ::"n"(32 * EPI) : "memory"); }
 
 // tcgen05.cp of a 32-row x 16-byte matrix (rows 16 bytes apart in shared memory) into 32 lanes x 4
 // columns of tensor memory, replicated to the four lane quadrants.
@@ -131,16 +138,19 @@ template <>
 __device__ __forceinline__ void tmem_ld_ch<16>(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld16(taddr, r); }
 
 template <int NQ, bool SAMPLE>
-__global__ void __launch_bounds__(kThr, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap tmap) {
+__global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap tmap) {
     using G = Cfg<NQ>;
-    extern __shared__ unsigned char smem_raw[];
-    unsigned char* sm = reinterpret_cast<unsigned char*>(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    // 1024-byte aligned by offsetting the shared array itself (not through an integer), so that the
+    // compiler keeps every access below in the shared state space
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     unsigned char* bq = sm;
     unsigned char* stg = sm + G::BQ;
     float* thr_s = reinterpret_cast<float*>(stg + kSt * kStageB);
     int* ql_s = reinterpret_cast<int*>(thr_s + NQ);
     unsigned int* cnt_s = reinterpret_cast<unsigned int*>(ql_s + NQ);
-    uint64_t* full = reinterpret_cast<uint64_t*>(cnt_s + NQ);
+    float* hstage = reinterpret_cast<float*>(cnt_s + NQ);  // [EPI warps][32 lanes][HS]
+    uint64_t* full = reinterpret_cast<uint64_t*>(hstage + G::EPI * 32 * G::HS);
     uint64_t* empty = full + kSt;
     uint64_t* dfull = empty + kSt;
     uint64_t* dfree = dfull + G::NSLOT;
@@ -268,7 +278,7 @@ __global__ void __launch_bounds__(kThr, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_
     } else {
         // ---- accumulator readers ----
         const int ew = warp - 2;
-        const int set = ew >> 2;                 // warps 2-5 and 6-9 take alternate slots
+        const int set = ew >> 2;                 // set u % SETS reads slot use u
         const int quad = warp & 3;               // the lane quadrant this warp may access
         const int et = tid - 64;                 // 0..255
         const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
@@ -293,14 +303,14 @@ __global__ void __launch_bounds__(kThr, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_
             const int chunk = SAMPLE ? 0 : t0 / P.kc;
             // the previous item's accumulators are all read (so its MMAs are done) before the query
             // tile and its scale factors are replaced
-            epi_sync();
-            for (int e = et; e < NQ * 8; e += 32 * kEpi) {
+            epi_sync<G::EPI>();
+            for (int e = et; e < NQ * 8; e += 32 * G::EPI) {
                 const int r = e >> 3, c = e & 7;
                 uint4 v = make_uint4(0, 0, 0, 0);
                 if (r < nrow) v = *reinterpret_cast<const uint4*>(qc + (size_t)(rbase + r) * kIKBytes + 16 * c);
                 *reinterpret_cast<uint4*>(bq + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) = v;
             }
-            for (int e = et; e < NQ; e += 32 * kEpi) {
+            for (int e = et; e < NQ; e += 32 * G::EPI) {
                 int ql = -1;
                 float th = __int_as_float(0x7f800000);
                 if (e < nrow) {
@@ -328,62 +338,97 @@ __global__ void __launch_bounds__(kThr, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_
             }
             fence_async_smem();
             tc_fence_before();
-            epi_sync();
+            epi_sync<G::EPI>();
             if (et == 0) mbar_arrive(qready);
             for (int k = 0; k < nt && !abort_s; ++k) {
                 const int t = SAMPLE ? mma_sample_tile(P.st, t0 + k) : t0 + k;
                 const int p = t * kTP + 32 * quad + lane;
                 for (int h = 0; h < G::H; ++h, ++u) {
-                    if ((u & 1) != set) continue;
+                    if (u % G::SETS != set) continue;
                     const int slot = u % G::NSLOT;
                     const uint32_t ph = (uint32_t)(u / G::NSLOT) & 1u;
                     const bool ok = __all_sync(0xffffffffu, mbar_wait(&dfull[slot], ph, kWaitNs));
                     if (!ok) { if (lane == 0) fail(); break; }
                     tc_fence_after();
-#pragma unroll 1
-                    for (int c0 = 0; c0 < G::W; c0 += G::CH) {
-                        uint32_t v[G::CH];
-                        tmem_ld_ch<G::CH>(tbase + lane_off + (uint32_t)(slot * G::W + c0), v);
-                        tmem_ld_wait();
-                        const int colb = h * G::W + c0;
-                        if (SAMPLE) {
-                            float x[G::CH];
+                    // sampling: the column maxima of one chunk of CH accumulator columns (queries)
+                    auto sample = [&](const uint32_t (&v)[G::CH], int colb) {
+                        float x[G::CH];
 #pragma unroll
-                            for (int i = 0; i < G::CH; ++i)
-                                x[i] = p <= ql_s[colb + i] ? __uint_as_float(v[i]) : -__int_as_float(0x7f800000);
-                            const float m = lane_col_max<G::CH>(x);
-                            const int col = colb + (lane % G::CH);
-                            if (lane < G::CH && ql_s[col] >= 0)
-                                atomicMax(&tm[(size_t)(rbase + col) * P.ns + (t0 + k)], f32_order(m));
-                        } else {
-                            // this thread's columns at or above their thresholds, as a bit mask
-                            uint32_t m = 0;
-                            const float4* t4 = reinterpret_cast<const float4*>(thr_s + colb);
+                        for (int i = 0; i < G::CH; ++i)
+                            x[i] = p <= ql_s[colb + i] ? __uint_as_float(v[i]) : -__int_as_float(0x7f800000);
+                        const float m = lane_col_max<G::CH>(x);
+                        const int col = colb + (lane % G::CH);
+                        if (lane < G::CH && ql_s[col] >= 0)
+                            atomicMax(&tm[(size_t)(rbase + col) * P.ns + (t0 + k)], f32_order(m));
+                    };
+                    // filtering: this thread's columns at or above their thresholds, as a bit mask
+                    // (independent 4-bit groups, then an OR tree: no serial dependency chain)
+                    auto hitmask = [&](const uint32_t (&v)[G::CH], int colb) -> uint32_t {
+                        const float4* t4 = reinterpret_cast<const float4*>(thr_s + colb);
+                        uint32_t mk[G::CH / 4];
 #pragma unroll
-                            for (int i4 = 0; i4 < G::CH / 4; ++i4) {
-                                const float4 tt = t4[i4];
-                                m |= (__uint_as_float(v[4 * i4 + 0]) >= tt.x ? 1u : 0u) << (4 * i4 + 0);
-                                m |= (__uint_as_float(v[4 * i4 + 1]) >= tt.y ? 1u : 0u) << (4 * i4 + 1);
-                                m |= (__uint_as_float(v[4 * i4 + 2]) >= tt.z ? 1u : 0u) << (4 * i4 + 2);
-                                m |= (__uint_as_float(v[4 * i4 + 3]) >= tt.w ? 1u : 0u) << (4 * i4 + 3);
+                        for (int i4 = 0; i4 < G::CH / 4; ++i4) {
+                            const float4 tt = t4[i4];
+                            const uint32_t g = (__uint_as_float(v[4 * i4 + 0]) >= tt.x ? 1u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 1]) >= tt.y ? 2u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 2]) >= tt.z ? 4u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 3]) >= tt.w ? 8u : 0u);
+                            mk[i4] = g << (4 * i4);
+                        }
+#pragma unroll
+                        for (int w = G::CH / 8; w >= 1; w >>= 1)
+#pragma unroll
+                            for (int i = 0; i < w; ++i) mk[i] |= mk[i + w];
+                        return mk[0];
+                    };
+                    // the admitted positions of one chunk go to their rows' lists of this item
+                    auto admit = [&](const uint32_t (&v)[G::CH], int colb, uint32_t m) {
+                        if (!m) return;
+                        // the values go through this lane's staging row, read back by index
+                        float* hs = hstage + ((size_t)ew * 32 + lane) * G::HS;
+#pragma unroll
+                        for (int i4 = 0; i4 < G::CH / 4; ++i4)
+                            *reinterpret_cast<float4*>(hs + 4 * i4) =
+                                make_float4(__uint_as_float(v[4 * i4]), __uint_as_float(v[4 * i4 + 1]),
+                                            __uint_as_float(v[4 * i4 + 2]), __uint_as_float(v[4 * i4 + 3]));
+                        do {
+                            const int i = __ffs(m) - 1;
+                            m &= m - 1;
+                            const int col = colb + i;
+                            if (p > ql_s[col]) continue;
+                            // this CTA alone fills the row's list of this item: a shared counter
+                            const unsigned int o = atomicAdd(&cnt_s[col], 1u);
+                            if (o < (unsigned)sub) {
+                                const size_t off = ((size_t)(rbase + col) * P.nchunks + chunk) * sub + o;
+                                cpos[off] = p;
+                                cval[off] = hs[i];
                             }
-                            while (m) {
-                                const int i = __ffs(m) - 1;
-                                m &= m - 1;
-                                const int col = colb + i;
-                                if (p > ql_s[col]) continue;
-                                float x = __uint_as_float(v[0]);
-#pragma unroll
-                                for (int q = 1; q < G::CH; ++q) x = (i == q) ? __uint_as_float(v[q]) : x;
-                                // this CTA alone fills the row's list of this item: a shared counter
-                                const unsigned int o = atomicAdd(&cnt_s[col], 1u);
-                                if (o < (unsigned)sub) {
-                                    const size_t off = ((size_t)(rbase + col) * P.nchunks + chunk) * sub + o;
-                                    cpos[off] = p;
-                                    cval[off] = x;
-                                }
+                        } while (m);
+                    };
+                    const uint32_t dcol = tbase + lane_off + (uint32_t)(slot * G::W);
+                    if (G::W >= 2 * G::CH) {
+#pragma unroll 1
+                        for (int c0 = 0; c0 < G::W; c0 += 2 * G::CH) {
+                            uint32_t v0[G::CH], v1[G::CH];
+                            tmem_ld_ch<G::CH>(dcol + (uint32_t)c0, v0);
+                            tmem_ld_ch<G::CH>(dcol + (uint32_t)(c0 + G::CH), v1);
+                            tmem_ld_wait();
+                            const int cb = h * G::W + c0;
+                            if (SAMPLE) {
+                                sample(v0, cb);
+                                sample(v1, cb + G::CH);
+                            } else {
+                                const uint32_t m0 = hitmask(v0, cb), m1 = hitmask(v1, cb + G::CH);
+                                admit(v0, cb, m0);
+                                admit(v1, cb + G::CH, m1);
                             }
                         }
+                    } else {
+                        uint32_t v0[G::CH];
+                        tmem_ld_ch<G::CH>(dcol, v0);
+                        tmem_ld_wait();
+                        if (SAMPLE) sample(v0, h * G::W);
+                        else admit(v0, h * G::W, hitmask(v0, h * G::W));
                     }
                     tc_fence_before();
                     __syncwarp();
@@ -392,8 +437,8 @@ __global__ void __launch_bounds__(kThr, Cfg<NQ>::COLS <= 256 ? 2 : 1) mma_score_
             }
             if (!SAMPLE) {
                 // the item's candidate counts (a count above subcap marks an overflowed list)
-                epi_sync();
-                for (int e = et; e < nrow; e += 32 * kEpi) cnt[(size_t)(rbase + e) * P.nchunks + chunk] = cnt_s[e];
+                epi_sync<G::EPI>();
+                for (int e = et; e < nrow; e += 32 * G::EPI) cnt[(size_t)(rbase + e) * P.nchunks + chunk] = cnt_s[e];
             }
         }
     }
@@ -535,17 +580,20 @@ cudaError_t launch_score(const IndexArgs& a, const CUtensorMap& map, int sms, cu
     auto k = mma_score_kernel<NQ, SAMPLE>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::SMEM);
     if (e != cudaSuccess) return e;
+    // the largest shared-memory carveout, so that two 16-column CTAs fit on an SM
+    e = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     const MmaPlan& P = a.plan.mma;
     const long long items = (long long)P.nseq * P.nqt * (SAMPLE ? P.nschunks : P.nchunks);
     int per_sm = 0;  // two CTAs share an SM's tensor memory when each takes 256 columns
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThr, G::SMEM);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, G::THREADS, G::SMEM);
     if (e != cudaSuccess) return e;
     if (per_sm > (G::COLS <= 256 ? 2 : 1)) per_sm = G::COLS <= 256 ? 2 : 1;
     if (per_sm < 1) per_sm = 1;
     long long grid = (long long)sms * per_sm;
     if (grid > items) grid = items;
     if (grid < 1) return cudaSuccess;
-    k<<<(unsigned)grid, kThr, G::SMEM, s>>>(a, map);
+    k<<<(unsigned)grid, G::THREADS, G::SMEM, s>>>(a, map);
     return cudaGetLastError();
 }
 

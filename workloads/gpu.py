@@ -69,13 +69,36 @@ class Step:
                                out_f32=out_f32, lse=lse, ws=ws, stream=stream)
         hooks("attend", 1)
 
+    def _prefill_parts(self, hooks, stream):
+        """The prefill chunk as the three calls csa2_prefill_chunk makes: append the chunk at
+        p0 = context - tq, index its tq rows (row i at position p0 + i), attend them."""
+        wl, I, O, t = self.wl, self.inputs, self.outputs, self.wl.tq
+        p0 = wl.context - t
+        dev = I["idx_q"].device
+        if not hasattr(self, "_pp"):
+            self._pp = (torch.full((1,), p0, dtype=torch.int64, device=dev),
+                        torch.arange(p0, wl.context, dtype=torch.int64, device=dev))
+        pos, qpos = self._pp
+        hooks("append", 0)
+        csa.csa2_quantize_append(self.shape, self.cache, 1, t, pos, I["kv"], I["idx_k"], I["swa_kv"], ws=self.ws,
+                                 stream=stream)
+        hooks("append", 1)
+        hooks("index", 0)
+        csa.csa2_index_topk_full(self.shape, self.cache, 1, t, qpos, I["idx_q"], wl.k, O["idx"], max_ctx=wl.context,
+                                 ws=self.ws, stream=stream)
+        hooks("index", 1)
+        hooks("attend", 0)
+        csa.csa2_sparse_attend(self.shape, self.cache, 1, t, qpos, I["q"], O["idx"], wl.k, O["out"], ws=self.ws,
+                               stream=stream)
+        hooks("attend", 1)
+
     # ---- the same pass as separate entry points (kernel-level timing) ----
     def run_parts(self, hooks, stream=None):
         """hooks(name) is called before and after each kernel's entry point: ('append'|'index'|'attend')."""
         wl, I, O = self.wl, self.inputs, self.outputs
         b = self.batch
         if wl.mode == "prefill":
-            raise NotImplementedError("prefill is timed through csa2_prefill_chunk")
+            return self._prefill_parts(hooks, stream)
         if wl.mode == "draft":
             return self._draft(hooks, stream, self.ws)
         hooks("append", 0)
