@@ -30,7 +30,7 @@
 //
 // Kernel roles (one CTA of 14 warps per SM with 256 query columns, two of 10 with 16): warp 0 issues
 // the TMA copies of key tiles (codes through a 128-byte-swizzled tensor map, scales by a bulk copy)
-// into a 4-stage ring; warp 1 turns the scales into tensor-core scale-factor matrices
+// into a ring of 4 stages (3 with 16 queries); warp 1 turns the scales into tensor-core scale-factor matrices
 // (tcgen05.cp, replicated over the four lane quadrants) and issues the MMAs into tensor-memory
 // accumulator slots; the other warps, in sets of four (one per lane quadrant) taking the slots in
 // turn, read the accumulators (tcgen05.ld) and either admit candidates or reduce tile maxima. A
@@ -50,7 +50,6 @@ namespace {
 using namespace tc;
 
 constexpr int kTP = kMmaTile;                  // key positions per tile (MMA M)
-constexpr int kSt = 4;                         // key tile stages
 constexpr int kCodeB = kTP * kIKBytes;         // 16384
 constexpr int kScB = kTP * kIKScales;          // 2048
 constexpr int kStageB = kCodeB + 2 * kScB;     // codes | raw scales | scale-factor matrices
@@ -59,21 +58,26 @@ constexpr float kEpsRel = 1.0f / 16384.0f;     // 2^-14
 
 template <int NQ>
 struct Cfg {
+    static constexpr int ST = NQ > 128 ? 4 : 3;     // key tile stages (two 16-query CTAs share an SM)
     static constexpr int W = NQ > 128 ? 128 : NQ;   // MMA N
     static constexpr int H = NQ / W;                // MMAs per K step
-    static constexpr int NSLOT = NQ > 128 ? 3 : 8;  // accumulator slots of W columns
+    static constexpr int TPS = NQ > 128 ? 1 : 4;    // key tiles per accumulator slot (W columns each)
+    static constexpr int SW = W * TPS;              // slot width in columns
+    static constexpr int NSLOT = NQ > 128 ? 3 : 2;  // accumulator slots
     static constexpr int SETS = NQ > 128 ? 3 : 2;   // sets of four accumulator-reading warps (one per
                                                     // lane quadrant); set u % SETS reads slot use u
     static constexpr int EPI = 4 * SETS;
     static constexpr int THREADS = 32 * (2 + EPI);
-    static constexpr int SFA = NSLOT * W;           // key scale factors: 16 columns per stage
-    static constexpr int SFB = SFA + 16 * kSt;      // query scale factors: 16 columns per half
+    static constexpr int SFA = NSLOT * SW;          // key scale factors: 16 columns per stage
+    static constexpr int SFB = SFA + 16 * ST;      // query scale factors: 16 columns per half
     static constexpr int COLS = SFB + 16 * H <= 256 ? 256 : 512;
     static constexpr int BQ = NQ * kIKBytes;        // query tile bytes
     static constexpr int CH = W < 32 ? W : 32;      // accumulator columns per tcgen05.ld
-    static constexpr int HS = CH + 4;               // floats per lane of a warp's hit staging rows
-    static constexpr size_t SMEM = 1024 + BQ + (size_t)kSt * kStageB + (size_t)NQ * 12 +
-                                   (size_t)EPI * 32 * HS * 4 + 8 * (2 * kSt + 2 * NSLOT + 2);
+    static constexpr int HS = (TPS > 1 ? 32 : CH) + 4;  // floats per lane of a warp's hit staging row
+                                                        // (one 32-column load; padded against bank
+                                                        // conflicts of its 16-byte stores)
+    static constexpr size_t SMEM = 1024 + BQ + (size_t)ST * kStageB + (size_t)NQ * 12 + 128 +
+                                   (size_t)EPI * 32 * HS * 4 + 8 * (2 * ST + 2 * NSLOT + 2);
 };
 
 template <int EPI>
@@ -146,13 +150,14 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
     unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     unsigned char* bq = sm;
     unsigned char* stg = sm + G::BQ;
-    float* thr_s = reinterpret_cast<float*>(stg + kSt * kStageB);
+    float* thr_s = reinterpret_cast<float*>(stg + G::ST * kStageB);
     int* ql_s = reinterpret_cast<int*>(thr_s + NQ);
     unsigned int* cnt_s = reinterpret_cast<unsigned int*>(ql_s + NQ);
-    float* hstage = reinterpret_cast<float*>(cnt_s + NQ);  // [EPI warps][32 lanes][HS]
+    float* thr2 = reinterpret_cast<float*>(cnt_s + NQ);     // 32 columns: thresholds of column % NQ
+    float* hstage = thr2 + 32;                              // [EPI warps][32 lanes][HS]
     uint64_t* full = reinterpret_cast<uint64_t*>(hstage + G::EPI * 32 * G::HS);
-    uint64_t* empty = full + kSt;
-    uint64_t* dfull = empty + kSt;
+    uint64_t* empty = full + G::ST;
+    uint64_t* dfull = empty + G::ST;
     uint64_t* dfree = dfull + G::NSLOT;
     uint64_t* qready = dfree + G::NSLOT;
     uint32_t* tslot = reinterpret_cast<uint32_t*>(qready + 1);
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
     uint32_t* status = reinterpret_cast<uint32_t*>(a.ws + kHdrStatus);
     const uint32_t* tend = reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_tend);
     if (tid == 0) {
-        for (int s = 0; s < kSt; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < G::ST; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
         for (int k = 0; k < G::NSLOT; ++k) { mbar_init(&dfull[k], 1); mbar_init(&dfree[k], 4); }
         mbar_init(qready, 1);
         abort_s = 0;
@@ -189,8 +194,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                 int b, j, t0, nt;
                 item_range<SAMPLE>(a, tend, it, b, j, t0, nt);
                 for (int k = 0; k < nt; ++k, ++kk) {
-                    const int s = kk % kSt;
-                    const uint32_t ph = (uint32_t)(kk / kSt) & 1u;
+                    const int s = kk % G::ST;
+                    const uint32_t ph = (uint32_t)(kk / G::ST) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u, kWaitNs)) { fail(); break; }
                     const int t = SAMPLE ? mma_sample_tile(P.st, t0 + k) : t0 + k;
                     const int64_t p0 = (int64_t)t * kTP;
@@ -204,8 +209,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                 }
             }
             // wait for the copies still in flight (all landed already unless a wait ran out)
-            for (int s = 0; s < kSt && s < kk; ++s) {
-                const int n = (kk - s + kSt - 1) / kSt;
+            for (int s = 0; s < G::ST && s < kk; ++s) {
+                const int n = (kk - s + G::ST - 1) / G::ST;
                 if (!mbar_wait(&full[s], (uint32_t)(n - 1) & 1u, kWaitNs)) set_status(status, CSA2_DEV_TIMEOUT);
             }
         }
@@ -225,8 +230,8 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
             if (!ok) { if (lane == 0) fail(); break; }
             tc_fence_after();
             for (int k = 0; k < nt; ++k, ++kk) {
-                const int s = kk % kSt;
-                const uint32_t ph = (uint32_t)(kk / kSt) & 1u;
+                const int s = kk % G::ST;
+                const uint32_t ph = (uint32_t)(kk / G::ST) & 1u;
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[s], ph, kWaitNs));
                 if (!ok) { if (lane == 0) fail(); break; }
                 unsigned char* st = stg + s * kStageB;
@@ -246,23 +251,30 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
 #pragma unroll
                     for (int q = 0; q < 4; ++q) tmem_cp_sf(sfa + 4 * q, smem_u32(sf) + 512 * q);
                 }
-                for (int h = 0; h < G::H; ++h, ++u) {
+                // slot use u takes the H halves of one tile (256 queries) or TPS consecutive tiles of
+                // an item (16 queries: tile k % TPS at column W * (k % TPS) of the slot)
+                const int sub = G::TPS > 1 ? k % G::TPS : 0;
+                const bool close = G::TPS == 1 || sub == G::TPS - 1 || k == nt - 1;
+                for (int h = 0; h < G::H; ++h) {
                     const int slot = u % G::NSLOT;
                     const uint32_t uph = (uint32_t)(u / G::NSLOT) & 1u;
-                    if (lane == 0) ok = mbar_wait(&dfree[slot], uph ^ 1u, kWaitNs);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
+                    if (sub == 0) {
+                        if (lane == 0) ok = mbar_wait(&dfree[slot], uph ^ 1u, kWaitNs);
+                        ok = __shfl_sync(0xffffffffu, ok, 0);
+                        if (!ok) break;
+                    }
                     if (lane == 0) {
                         tc_fence_after();
-                        const uint32_t d = tbase + (uint32_t)(slot * G::W);
+                        const uint32_t d = tbase + (uint32_t)(slot * G::SW + sub * G::W);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const uint64_t ad = sw128_desc(smem_u32(st) + 32 * q);
                             const uint64_t bd = sw128_desc(smem_u32(bq + h * G::W * kIKBytes) + 32 * q);
                             mma_mxf4(d, ad, bd, idesc, sfa + 4 * q, tbase + (uint32_t)(G::SFB + 16 * h + 4 * q), q > 0);
                         }
-                        mma_commit(&dfull[slot]);
+                        if (close) mma_commit(&dfull[slot]);
                     }
+                    if (close) ++u;
                 }
                 if (lane == 0) mma_commit(&empty[s]);
                 last_s = s;
@@ -322,6 +334,14 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                 thr_s[e] = th;
                 cnt_s[e] = 0;
             }
+            if (G::TPS > 1 && !SAMPLE) {  // a 32-column load spans 32 / NQ tiles of the same queries
+                for (int e = et; e < 32; e += 32 * G::EPI) {
+                    const int c = e % NQ;
+                    float th = __int_as_float(0x7f800000);
+                    if (c < nrow && index_row_last(a, rbase + c) >= 0) th = rowp[rbase + c].z;
+                    thr2[e] = th;
+                }
+            }
             if (set < G::H) {
                 // query scale factors of half `set`: column 4q + g, lane l <- scale word q of row l + 32 g
                 uint32_t w[16];
@@ -340,9 +360,10 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
             tc_fence_before();
             epi_sync<G::EPI>();
             if (et == 0) mbar_arrive(qready);
-            for (int k = 0; k < nt && !abort_s; ++k) {
+            for (int k = 0; k < nt && !abort_s; k += G::TPS) {
                 const int t = SAMPLE ? mma_sample_tile(P.st, t0 + k) : t0 + k;
                 const int p = t * kTP + 32 * quad + lane;
+                const int ng = min(G::TPS, nt - k);  // tiles in this slot use
                 for (int h = 0; h < G::H; ++h, ++u) {
                     if (u % G::SETS != set) continue;
                     const int slot = u % G::NSLOT;
@@ -381,6 +402,24 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                             for (int i = 0; i < w; ++i) mk[i] |= mk[i + w];
                         return mk[0];
                     };
+                    auto hitmask2 = [&](const uint32_t (&v)[32]) -> uint32_t {
+                        const float4* t4 = reinterpret_cast<const float4*>(thr2);
+                        uint32_t mk[8];
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 tt = t4[i4];
+                            const uint32_t g = (__uint_as_float(v[4 * i4 + 0]) >= tt.x ? 1u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 1]) >= tt.y ? 2u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 2]) >= tt.z ? 4u : 0u) |
+                                               (__uint_as_float(v[4 * i4 + 3]) >= tt.w ? 8u : 0u);
+                            mk[i4] = g << (4 * i4);
+                        }
+#pragma unroll
+                        for (int w = 4; w >= 1; w >>= 1)
+#pragma unroll
+                            for (int i = 0; i < w; ++i) mk[i] |= mk[i + w];
+                        return mk[0];
+                    };
                     // the admitted positions of one chunk go to their rows' lists of this item
                     auto admit = [&](const uint32_t (&v)[G::CH], int colb, uint32_t m) {
                         if (!m) return;
@@ -405,8 +444,61 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                             }
                         } while (m);
                     };
-                    const uint32_t dcol = tbase + lane_off + (uint32_t)(slot * G::W);
-                    if (G::W >= 2 * G::CH) {
+                    const uint32_t dcol = tbase + lane_off + (uint32_t)(slot * G::SW);
+                    if (G::TPS > 1) {
+                        // TPS tiles of W = 16 queries: column c <-> tile k + c / 16, query c % 16
+                        static_assert(G::TPS == 1 || (G::W == 16 && G::TPS == 4), "grouped slots: 4 tiles x 16");
+                        uint32_t v0[32], v1[32];
+                        tmem_ld32(dcol, v0);
+                        tmem_ld32(dcol + 32u, v1);
+                        tmem_ld_wait();
+                        // key position of this thread in tile k + sb
+                        auto pos_of = [&](int sb) {
+                            const int tt = SAMPLE ? mma_sample_tile(P.st, t0 + k + sb) : t0 + k + sb;
+                            return tt * kTP + 32 * quad + lane;
+                        };
+                        auto grouped = [&](const uint32_t (&v)[32], int c) {  // tiles 2c, 2c + 1
+                            const int pa = pos_of(2 * c), pb = pos_of(2 * c + 1);
+                            const bool va = 2 * c < ng, vb = 2 * c + 1 < ng;
+                            if (SAMPLE) {
+                                float x[32];
+#pragma unroll
+                                for (int i = 0; i < 32; ++i) {
+                                    const bool ok2 = i < 16 ? (va && pa <= ql_s[i & 15]) : (vb && pb <= ql_s[i & 15]);
+                                    x[i] = ok2 ? __uint_as_float(v[i]) : -__int_as_float(0x7f800000);
+                                }
+                                const float m = lane_col_max<32>(x);
+                                const int q = lane & 15, sb = 2 * c + (lane >> 4);
+                                if (sb < ng && ql_s[q] >= 0)
+                                    atomicMax(&tm[(size_t)(rbase + q) * P.ns + (t0 + k + sb)], f32_order(m));
+                            } else {
+                                uint32_t m = hitmask2(v);
+                                m &= (va ? 0x0000FFFFu : 0u) | (vb ? 0xFFFF0000u : 0u);
+                                if (!m) return;
+                                float* hs = hstage + ((size_t)ew * 32 + lane) * G::HS;
+#pragma unroll
+                                for (int i4 = 0; i4 < 8; ++i4)
+                                    *reinterpret_cast<float4*>(hs + 4 * i4) =
+                                        make_float4(__uint_as_float(v[4 * i4]), __uint_as_float(v[4 * i4 + 1]),
+                                                    __uint_as_float(v[4 * i4 + 2]), __uint_as_float(v[4 * i4 + 3]));
+                                do {
+                                    const int i = __ffs(m) - 1;
+                                    m &= m - 1;
+                                    const int q = i & 15;
+                                    const int pp = i < 16 ? pa : pb;
+                                    if (pp > ql_s[q]) continue;
+                                    const unsigned int o = atomicAdd(&cnt_s[q], 1u);
+                                    if (o < (unsigned)sub) {
+                                        const size_t off = ((size_t)(rbase + q) * P.nchunks + chunk) * sub + o;
+                                        cpos[off] = pp;
+                                        cval[off] = hs[i];
+                                    }
+                                } while (m);
+                            }
+                        };
+                        grouped(v0, 0);
+                        if (ng > 2) grouped(v1, 1);
+                    } else if (G::W >= 2 * G::CH) {
 #pragma unroll 1
                         for (int c0 = 0; c0 < G::W; c0 += 2 * G::CH) {
                             uint32_t v0[G::CH], v1[G::CH];
@@ -585,11 +677,13 @@ cudaError_t launch_score(const IndexArgs& a, const CUtensorMap& map, int sms, cu
     if (e != cudaSuccess) return e;
     const MmaPlan& P = a.plan.mma;
     const long long items = (long long)P.nseq * P.nqt * (SAMPLE ? P.nschunks : P.nchunks);
-    int per_sm = 0;  // two CTAs share an SM's tensor memory when each takes 256 columns
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, G::THREADS, G::SMEM);
+    int fit = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, k, G::THREADS, G::SMEM);
     if (e != cudaSuccess) return e;
-    if (per_sm > (G::COLS <= 256 ? 2 : 1)) per_sm = G::COLS <= 256 ? 2 : 1;
-    if (per_sm < 1) per_sm = 1;
+    if (fit < 1) return cudaErrorInvalidConfiguration;
+    // two CTAs share an SM's tensor memory when each takes 256 columns; their registers (launch
+    // bounds) and shared memory (with the largest carveout) are sized for two per SM
+    const int per_sm = G::COLS <= 256 ? 2 : 1;
     long long grid = (long long)sms * per_sm;
     if (grid > items) grid = items;
     if (grid < 1) return cudaSuccess;
