@@ -572,6 +572,7 @@ __global__ void __launch_bounds__(256) mma_prep_kernel(const IndexArgs a, int qb
     if (n > a.c.cap) n = a.c.cap;
     const uint4* sc = reinterpret_cast<const uint4*>(a.c.ik_scale + (size_t)b * a.c.cap * kIKScales);
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+#pragma unroll 4
     for (int64_t p = (int64_t)part * 256 + tid; p < n; p += (int64_t)sblocks * 256) {
         const uint4 v = __ldg(sc + p);
         m0 = __vmaxu4(m0, v.x & 0x7F7F7F7Fu);
