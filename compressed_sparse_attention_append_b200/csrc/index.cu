@@ -717,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 3) mma_final_kernel(IndexArgs a) {
     __shared__ unsigned int hist[256];
     __shared__ int kf_lut[256];
     __shared__ unsigned int nabove, nsel, bad, ntot;
-    __shared__ unsigned int coff[256];
+    __shared__ unsigned int coff[256], ccnt[256];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int row = blockIdx.x, K = a.plan.k;
     const MmaPlan& P = a.plan.mma;
@@ -756,11 +756,14 @@ __global__ void __launch_bounds__(kThreads, 3) mma_final_kernel(IndexArgs a) {
         const int te = (int)reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_tend)[b * P.nqt + j];
         const int nch = (te + P.kc - 1) / P.kc;
         const uint32_t* cc = reinterpret_cast<const uint32_t*>(a.ws + a.L.mma_cnt) + (size_t)row * P.nchunks;
+        // every list's count into shared memory in one pass, then their offsets
+        for (int c = tid; c < nch && c < 256; c += kThreads) ccnt[c] = cc[c];
+        __syncthreads();
         if (warp == 0) {
             unsigned int run = 0;
             for (int c0 = 0; c0 < nch; c0 += 32) {
                 const int c = c0 + lane;
-                const unsigned int v = c < nch ? cc[c] : 0u;
+                const unsigned int v = (c < nch && c < 256) ? ccnt[c] : 0u;
                 if (v > (unsigned)P.subcap) atomicOr(&bad, 1u);
                 unsigned int incl = v;
 #pragma unroll
@@ -780,15 +783,21 @@ __global__ void __launch_bounds__(kThreads, 3) mma_final_kernel(IndexArgs a) {
             const int* cp = reinterpret_cast<const int*>(a.ws + a.L.mma_cpos) + (size_t)row * P.nchunks * P.subcap;
             const uint32_t otau = f32_order(tau);
             unsigned int above = 0;
-            for (int c = warp; c < nch; c += kWarps) {  // one warp per list
-                const int m = (int)cc[c];
-                const size_t src = (size_t)c * P.subcap;
-                for (int i = lane; i < m; i += 32) {
-                    const uint32_t o = f32_order(cv[src + i]);
-                    ckey[coff[c] + i] = o;
-                    cposs[coff[c] + i] = cp[src + i];
-                    above += o >= otau;
+            // candidate o of the row: list c = the last one starting at or before o (binary search
+            // over the offsets); every thread's loads are independent of one another
+            const int tot = (int)ntot;
+#pragma unroll 4
+            for (int o = tid; o < tot; o += kThreads) {
+                int lo = 0, hi = nch - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if ((int)coff[mid] <= o) lo = mid; else hi = mid - 1;
                 }
+                const size_t src = (size_t)lo * P.subcap + (o - (int)coff[lo]);
+                const uint32_t k2 = f32_order(cv[src]);
+                ckey[o] = k2;
+                cposs[o] = cp[src];
+                above += k2 >= otau;
             }
             above = __reduce_add_sync(0xffffffffu, above);
             if (lane == 0 && above) atomicAdd(&nabove, above);
