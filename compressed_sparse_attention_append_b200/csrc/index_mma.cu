@@ -76,7 +76,7 @@ struct Cfg {
     static constexpr int HS = (TPS > 1 ? 32 : CH) + 4;  // floats per lane of a warp's hit staging row
                                                         // (one 32-column load; padded against bank
                                                         // conflicts of its 16-byte stores)
-    static constexpr size_t SMEM = 1024 + BQ + (size_t)ST * kStageB + (size_t)NQ * 12 + 128 +
+    static constexpr size_t SMEM = 1024 + BQ + (size_t)ST * kStageB + (size_t)NQ * 12 + 128 + (NQ < 32 ? 64 : NQ * 2) +
                                    (size_t)EPI * 32 * HS * 4 + 8 * (2 * ST + 2 * NSLOT + 2);
 };
 
@@ -154,7 +154,10 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
     int* ql_s = reinterpret_cast<int*>(thr_s + NQ);
     unsigned int* cnt_s = reinterpret_cast<unsigned int*>(ql_s + NQ);
     float* thr2 = reinterpret_cast<float*>(cnt_s + NQ);     // 32 columns: thresholds of column % NQ
-    float* hstage = thr2 + 32;                              // [EPI warps][32 lanes][HS]
+    // thresholds rounded down to fp16, paired for the packed test: entry 16 g + p of a 32-column
+    // load holds columns 32 g + p and 32 g + p + 16
+    __half2* thh = reinterpret_cast<__half2*>(thr2 + 32);
+    float* hstage = reinterpret_cast<float*>(thh + (NQ < 32 ? 16 : NQ / 2));  // [EPI warps][32 lanes][HS]
     uint64_t* full = reinterpret_cast<uint64_t*>(hstage + G::EPI * 32 * G::HS);
     uint64_t* empty = full + G::ST;
     uint64_t* dfull = empty + G::ST;
@@ -342,6 +345,17 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                     thr2[e] = th;
                 }
             }
+            if (!SAMPLE) {
+                constexpr int NP = NQ < 32 ? 16 : NQ / 2;
+                for (int e = et; e < NP; e += 32 * G::EPI) {
+                    const int g = e >> 4, pp = e & 15;
+                    const int c0 = (32 * g + pp) % NQ, c1 = (32 * g + pp + 16) % NQ;
+                    float t0 = __int_as_float(0x7f800000), t1 = t0;
+                    if (c0 < nrow && index_row_last(a, rbase + c0) >= 0) t0 = rowp[rbase + c0].z;
+                    if (c1 < nrow && index_row_last(a, rbase + c1) >= 0) t1 = rowp[rbase + c1].z;
+                    thh[e] = __halves2half2(__float2half_rd(t0), __float2half_rd(t1));
+                }
+            }
             if (set < G::H) {
                 // query scale factors of half `set`: column 4q + g, lane l <- scale word q of row l + 32 g
                 uint32_t w[16];
@@ -384,7 +398,21 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                     };
                     // filtering: this thread's columns at or above their thresholds, as a bit mask
                     // (independent 4-bit groups, then an OR tree: no serial dependency chain)
+                    // A superset test in fp16: values p and p + 16 of a 32-column load are packed and
+                    // compared with thresholds rounded down (a value at or above its fp32 threshold
+                    // rounds to at least the rounded-down threshold); admitted values are checked
+                    // again exactly. Four independent partial masks.
+                    auto packed_mask = [&](const uint32_t (&v)[32], const __half2* th) -> uint32_t {
+                        uint32_t mk[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                        for (int pp = 0; pp < 16; ++pp) {
+                            const __half2 hv = __floats2half2_rn(__uint_as_float(v[pp]), __uint_as_float(v[pp + 16]));
+                            mk[pp & 3] |= __hge2_mask(hv, th[pp]) & (0x00010001u << pp);
+                        }
+                        return (mk[0] | mk[1]) | (mk[2] | mk[3]);
+                    };
                     auto hitmask = [&](const uint32_t (&v)[G::CH], int colb) -> uint32_t {
+                        if constexpr (G::CH == 32) return packed_mask(v, thh + (colb >> 5) * 16);
                         const float4* t4 = reinterpret_cast<const float4*>(thr_s + colb);
                         uint32_t mk[G::CH / 4];
 #pragma unroll
@@ -402,24 +430,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                             for (int i = 0; i < w; ++i) mk[i] |= mk[i + w];
                         return mk[0];
                     };
-                    auto hitmask2 = [&](const uint32_t (&v)[32]) -> uint32_t {
-                        const float4* t4 = reinterpret_cast<const float4*>(thr2);
-                        uint32_t mk[8];
-#pragma unroll
-                        for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 tt = t4[i4];
-                            const uint32_t g = (__uint_as_float(v[4 * i4 + 0]) >= tt.x ? 1u : 0u) |
-                                               (__uint_as_float(v[4 * i4 + 1]) >= tt.y ? 2u : 0u) |
-                                               (__uint_as_float(v[4 * i4 + 2]) >= tt.z ? 4u : 0u) |
-                                               (__uint_as_float(v[4 * i4 + 3]) >= tt.w ? 8u : 0u);
-                            mk[i4] = g << (4 * i4);
-                        }
-#pragma unroll
-                        for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                            for (int i = 0; i < w; ++i) mk[i] |= mk[i + w];
-                        return mk[0];
-                    };
+                    auto hitmask2 = [&](const uint32_t (&v)[32]) -> uint32_t { return packed_mask(v, thh); };
                     // the admitted positions of one chunk go to their rows' lists of this item
                     auto admit = [&](const uint32_t (&v)[G::CH], int colb, uint32_t m) {
                         if (!m) return;
@@ -434,7 +445,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                             const int i = __ffs(m) - 1;
                             m &= m - 1;
                             const int col = colb + i;
-                            if (p > ql_s[col]) continue;
+                            if (p > ql_s[col] || !(hs[i] >= thr_s[col])) continue;
                             // this CTA alone fills the row's list of this item: a shared counter
                             const unsigned int o = atomicAdd(&cnt_s[col], 1u);
                             if (o < (unsigned)sub) {
@@ -486,7 +497,7 @@ __global__ void __launch_bounds__(Cfg<NQ>::THREADS, Cfg<NQ>::COLS <= 256 ? 2 : 1
                                     m &= m - 1;
                                     const int q = i & 15;
                                     const int pp = i < 16 ? pa : pb;
-                                    if (pp > ql_s[q]) continue;
+                                    if (pp > ql_s[q] || !(hs[i] >= thr2[i])) continue;
                                     const unsigned int o = atomicAdd(&cnt_s[q], 1u);
                                     if (o < (unsigned)sub) {
                                         const size_t off = ((size_t)(rbase + q) * P.nchunks + chunk) * sub + o;
