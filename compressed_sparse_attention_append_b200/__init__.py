@@ -48,7 +48,7 @@ EXPORTS = (
     "csa2_entry_bytes", "csa2_status_string", "csa2_version", "csa2_workspace_size", "csa2_workspace_init",
     "csa2_quantize_append", "csa2_index_topk_full", "csa2_index_topk_reindex", "csa2_sparse_attend",
     "csa2_decode_full", "csa2_decode_reindex", "csa2_decode_minimal", "csa2_prefill_chunk",
-    "csa2_get_device_status", "csa2_sparse_attend_noalloc",
+    "csa2_get_device_status", "csa2_sparse_attend_noalloc", "csa2_mx_entry_bytes", "csa2_mxfp4_quantize",
 )
 
 
@@ -98,6 +98,8 @@ def lib():
             "csa2_prefill_chunk": (i, [S, C, i64, i, vp, vp, vp, vp, vp, i, vp, i64, f, vp, vp, vp, u32, vp, sz, vp]),
             "csa2_get_device_status": (i, [vp, vp, ctypes.POINTER(ctypes.c_int32)]),
             "csa2_sparse_attend_noalloc": (i, [S, C, i, i, vp, vp, vp, i, vp, f, vp, vp, vp, vp]),
+            "csa2_mx_entry_bytes": (sz, [i]),
+            "csa2_mxfp4_quantize": (i, [vp, i64, i, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -146,6 +148,11 @@ def _f32(t):
     return _typed(t, torch.float32)
 
 
+def _u8(t):
+    """byte outputs (codes, E8M0 scales): pointer only, after a dtype check."""
+    return _typed(t, torch.uint8)
+
+
 def _bits(t):
     """bf16 tensors travel as their 16-bit patterns; pointer only."""
     if t is None:
@@ -186,6 +193,16 @@ class Cache:
 
 def csa2_entry_bytes(channels: int) -> int:
     return lib().csa2_entry_bytes(int(channels))
+
+
+def csa2_mx_entry_bytes(channels: int) -> int:
+    return lib().csa2_mx_entry_bytes(int(channels))
+
+
+def csa2_mxfp4_quantize(x, data, scale, stream=None):
+    """MXFP4 rows: x [rows, channels] bf16 -> data [rows, channels/2] u8, scale [rows, channels/32] u8."""
+    rows, ch = x.shape
+    _check("csa2_mxfp4_quantize", lib().csa2_mxfp4_quantize(_bits(x), rows, ch, _u8(data), _u8(scale), _stream(stream)))
 
 
 def csa2_status_string(s: int) -> str:

@@ -168,6 +168,19 @@ size_t csa2_entry_bytes(int channels) {
     return (size_t)channels / 2 + (size_t)channels / 16;
 }
 
+size_t csa2_mx_entry_bytes(int channels) {
+    if (channels <= 0 || channels % 32) return 0;
+    return (size_t)channels / 2 + (size_t)channels / 32;
+}
+
+csa2_status csa2_mxfp4_quantize(const uint16_t* x, int64_t rows, int channels, uint8_t* data, uint8_t* scale,
+                                void* stream) {
+    if (rows < 0 || channels <= 0 || channels % 32 || !x || !data || !scale || !al16(x) || !al16(data))
+        return CSA2_ERR_INVALID_ARG;
+    if (rows == 0) return CSA2_OK;
+    return from_cuda(launch_mxfp4(x, (long long)rows, channels, data, scale, (cudaStream_t)stream));
+}
+
 const char* csa2_status_string(csa2_status s) {
     switch (s) {
         case CSA2_OK: return "ok";

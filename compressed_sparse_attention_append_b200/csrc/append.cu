@@ -72,7 +72,54 @@ __global__ void __launch_bounds__(192) append_kernel(AppendArgs a) {
     }
 }
 
+// MXFP4 rows ([C] sec. VII): one thread per 32-channel block. X = 2^(floor(log2 amax) - 2), byte
+// log2 X + 127 clamped to 0..254; x / X is exact (a power-of-two scale), so the hardware E2M1
+// conversion of the fp32 quotient decides each code as an exact rational would.
+__global__ void __launch_bounds__(256) mxfp4_kernel(const uint16_t* x, long long blocks, int nb, uint8_t* data,
+                                                    uint8_t* scale) {
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= blocks) return;
+    const uint4* src = reinterpret_cast<const uint4*>(x + id * 32);
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 v = __ldg(src + i);
+        w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[i] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(w[i] & 0xFFFF0000u)));
+    }
+    int sb = 0;
+    if (amax > 0.f) {
+        sb = ilogbf(amax) - 2 + 127;  // floor(log2 amax), subnormals included
+        sb = sb < 0 ? 0 : (sb > 254 ? 254 : sb);
+    }
+    uint32_t c[4] = {0u, 0u, 0u, 0u};
+    if (amax > 0.f) {
+        const float X = ldexpf(1.0f, sb - 127);  // 2^-127 .. 2^127, exact in fp32
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float lo = __fdiv_rn(__uint_as_float(w[i] << 16), X);
+            const float hi = __fdiv_rn(__uint_as_float(w[i] & 0xFFFF0000u), X);
+            c[i >> 2] |= f32x2_to_e2m1x2(lo, hi) << (8 * (i & 3));
+        }
+    }
+    *reinterpret_cast<uint4*>(data + id * 16) = make_uint4(c[0], c[1], c[2], c[3]);
+    scale[id] = (uint8_t)sb;
+}
+
 }  // namespace
+
+cudaError_t launch_mxfp4(const uint16_t* x, long long rows, int channels, uint8_t* data, uint8_t* scale,
+                         cudaStream_t s) {
+    const long long blocks = rows * (channels / 32);
+    if (blocks == 0) return cudaSuccess;
+    mxfp4_kernel<<<(unsigned)((blocks + 255) / 256), 256, 0, s>>>(x, blocks, channels / 32, data, scale);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s) {
     const long long threads = (long long)a.batch * a.t * 48;

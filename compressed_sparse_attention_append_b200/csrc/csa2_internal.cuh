@@ -412,6 +412,8 @@ struct AppendArgs {
     uint32_t* status;
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
+cudaError_t launch_mxfp4(const uint16_t* x, long long rows, int channels, uint8_t* data, uint8_t* scale,
+                         cudaStream_t s);  // append.cu: MXFP4 rows
 
 struct IndexArgs {
     csa2_cache c;

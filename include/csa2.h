@@ -105,6 +105,11 @@ typedef struct {
  * multiple of 16. Host only. */
 CSA2_API size_t csa2_entry_bytes(int channels);
 
+/* [C] sec. VII: an MXFP4 entry of `channels` E2M1 values with one 1-byte E8M0 scale per 32
+ * channels (the pages' indexer-key format) occupies channels/2 + channels/32 bytes. Returns 0 if
+ * channels is not a positive multiple of 32. Host only. */
+CSA2_API size_t csa2_mx_entry_bytes(int channels);
+
 /* Text of a status code. Host only; never NULL. */
 CSA2_API const char* csa2_status_string(csa2_status s);
 
@@ -270,6 +275,23 @@ CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* shape, const c
                                                 const int64_t* qpos, const uint16_t* q, const int32_t* idx, int k,
                                                 const int64_t* swa_begin, float sm_scale, uint16_t* out,
                                                 float* out_f32, float* lse, void* stream);
+
+/*
+ * MXFP4 row codec: the indexer-key format of the pages' own shape ([C] sec. VII names MXFP4: E2M1
+ * elements with one E8M0 scale per 32 channels). Rows of `channels` bf16 values (a positive
+ * multiple of 32) are quantised independently:
+ *   x     [rows][channels] bf16 (device, 16-byte aligned)
+ *   data  [rows][channels/2] E2M1 codes, channel 2j in the low nibble of byte j (device, 16-byte
+ *         aligned, caller-owned; a cache plane of such rows is data + position * channels/2)
+ *   scale [rows][channels/32] E8M0 bytes (device, caller-owned)
+ * Rule (the reading taken here; the pages name the format only): per 32-channel block with
+ * amax = max |x| > 0, the scale is X = 2^(floor(log2 amax) - 2) (6 = 1.5 * 2^2 is E2M1's largest
+ * value), stored as the byte log2 X + 127 clamped to 0..254; code_i = E2M1_RNE_satfinite(x_i / X)
+ * keeping the sign of x_i. amax == 0 gives scale byte 0 and all codes +0.
+ * Returns CSA2_ERR_INVALID_ARG for a null or misaligned pointer, rows < 0 or a bad `channels`.
+ */
+CSA2_API csa2_status csa2_mxfp4_quantize(const uint16_t* x, int64_t rows, int channels, uint8_t* data, uint8_t* scale,
+                                         void* stream);
 
 /* Synchronises `stream`, then reads and clears the device status word in `ws`.
  * *host_status receives the CSA2_DEV_* bits; returns CSA2_ERR_DEVICE if any bit was set. */

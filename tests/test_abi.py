@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_symbols()
-    assert len(names) == 15
+    assert len(names) == 17
     assert set(names) == set(csa.EXPORTS)
     for n in names:
         assert hasattr(L, n), n
@@ -224,3 +224,21 @@ def test_binding_checks_integer_and_float_dtypes(L):
         with pytest.raises(AssertionError, match="CUDA"):
             fn(torch.zeros(2, dtype=good))
         assert fn(None) is None
+
+
+def test_mx_entry_bytes_and_codec_validation(L):
+    """[C] sec. VII: an MXFP4 entry of ch channels is ch/2 + ch/32 bytes (the pages' 128-channel
+    indexer key: 68 B); the codec rejects bad arguments before any launch."""
+    assert csa.csa2_mx_entry_bytes(128) == 68
+    assert csa.csa2_mx_entry_bytes(512) == 272
+    assert csa.csa2_mx_entry_bytes(32) == 17
+    for bad in (0, 16, 48, -32):
+        assert csa.csa2_mx_entry_bytes(bad) == 0
+    f = L.csa2_mxfp4_quantize
+    buf = ctypes.create_string_buffer(4096 + 16)
+    base = (ctypes.addressof(buf) + 15) & ~15
+    assert f(None, 1, 32, base, base, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(base, 1, 48, base, base, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(base, -1, 32, base, base, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(base + 2, 1, 32, base, base, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(base, 0, 32, base, base, None) == csa.CSA2_OK  # nothing to do, no launch

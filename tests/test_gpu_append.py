@@ -128,3 +128,53 @@ def test_full_cache_fill_matches_oracle():
     for name in ("kv_data", "kv_scale", "ik_data", "ik_scale"):
         assert np.array_equal(getattr(cache, name)[1].cpu().numpy(), getattr(oc, name))
     assert np.array_equal(cache.swa[1, :5000].cpu().numpy(), oc.swa[:5000])
+
+
+def _mx_gpu(x_cpu, ch):
+    rows = x_cpu.shape[0]
+    data = torch.empty(rows, ch // 2, dtype=torch.uint8, device=DEV)
+    scale = torch.empty(rows, ch // 32, dtype=torch.uint8, device=DEV)
+    csa.csa2_mxfp4_quantize(x_cpu.to(DEV).contiguous(), data, scale)
+    return data.cpu().numpy(), scale.cpu().numpy()
+
+
+@pytest.mark.parametrize("ch,sigma", [(128, 1.0), (128, 8.0), (512, 1.0), (32, 1e-3), (128, 1e-38)])
+def test_mxfp4_codec_matches_oracle(orc, ch, sigma):
+    """The MXFP4 row codec of the pages' indexer key (E2M1 + E8M0 per 32 channels) against the
+    oracle's R13 codec, byte for byte: unit, large (clipped), small and subnormal values."""
+    rows = 2048
+    x = values(21, "ik", [0], torch.arange(rows), ch, "cpu", sigma)[0]
+    d, s = _mx_gpu(x, ch)
+    rd, rs = oracle.mx_quantize_rows(bf16_np(x), ch)
+    assert np.array_equal(s, rs)
+    assert np.array_equal(d, rd)
+
+
+def test_mxfp4_codec_every_value_at_many_scales(orc):
+    """Every finite bf16 value of magnitude <= A, in blocks whose largest magnitude is A, for block
+    maxima across the whole exponent range (subnormal and the largest included), so that every
+    E8M0 byte the rule can give and every E2M1 rounding decision is taken on the GPU and in the
+    oracle; plus all-zero and signed-zero blocks (byte 0, +0 codes)."""
+    pats = np.arange(0x10000, dtype=np.uint32).astype(np.uint16)
+    vals = pats.view(np.int16).astype(np.int32)
+    finite = (pats & 0x7F80) != 0x7F80
+    f32 = (pats.astype(np.uint32) << 16).view(np.float32)
+    blocks = []
+    for amax_bits in (0x0001, 0x0040, 0x0080, 0x00C0, 0x1234, 0x3F80, 0x3FC0, 0x40C0, 0x4B00, 0x7F7F):
+        A = np.float32((np.uint32(amax_bits) << 16).view(np.float32))
+        sel = pats[finite & (np.abs(f32) <= A)]
+        n = (len(sel) + 30) // 31
+        sel = np.resize(sel, n * 31)
+        blk = np.concatenate([np.full((n, 1), amax_bits, np.uint16), sel.reshape(n, 31)], axis=1)
+        blocks.append(blk)
+    nb = sum(b.shape[0] for b in blocks)
+    pad = (-(nb + 2)) % 4  # whole 128-channel rows
+    blocks.append(np.full((pad + 1, 32), 0x0000, np.uint16))
+    blocks.append(np.full((1, 32), 0x8000, np.uint16))
+    x = np.concatenate(blocks, axis=0).reshape(-1, 128)
+    xt = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16)
+    d, s = _mx_gpu(xt, 128)
+    rd, rs = oracle.mx_quantize_rows(x, 128)
+    assert np.array_equal(s, rs)
+    assert np.array_equal(d, rd)
+    assert (s.reshape(-1)[-2:] == 0).all() and (d.reshape(-1, 16)[-2:] == 0).all()
