@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(W * 32, (W == 8 ? 2 : 1)) attend_kernel(Attend
         }
     };
     if (W == 16) {
-        // round 1: warps 8..15 stage, warps 0..7 fold their partner's (m, l, O) into their own
+        // first merge step: warps 8..15 stage, warps 0..7 fold their partner's (m, l, O) into their own
         if (warp >= 8) stage_out(warp - 8);
         __syncthreads();
         if (warp < 8) {
