@@ -36,6 +36,10 @@ def algorithmic_bytes(wl):
     """Per query: dict kernel -> bytes. Entry sizes: FP4 main row 128 + 16 B, indexer row 128 + 16 B,
     window row 256 B (FP8)."""
     k, win = wl.k, wl.win
+    if wl.mode == "latent":
+        # the pages' own shape: k selected latent entries (256 B codes + 32 B scales), the window rows
+        # (512 B), the query and the output (64 heads x 512, bf16) and the indices, per row
+        return {"append": 0, "index": 0, "attend": k * 288 + win * 512 + 2 * (64 * 512 * 2) + k * 4}
     q, out, iq, idx = 16 * 128 * 2, 16 * 128 * 2, 4 * 64 * 2, k * 4
     attend = k * 144 + win * 256 + q + idx + out
     if wl.mode == "reindex":
@@ -61,6 +65,12 @@ def algorithmic_bytes(wl):
 L2_BYTES = 126 * 1024 * 1024
 
 
+def latent_flops(wl):
+    """Tensor work of one latent row: S^T = L Q^T and O^T = L^T P^T over k + win keys, 64 heads and
+    512 channels (2 flops per multiply-add)."""
+    return 2 * 2 * 64 * 512 * (wl.k + wl.win)
+
+
 def tensor_core_index(wl):
     """Several rows per sequence at a context of 8,192 or more (and k <= 1024) take the tensor-core
     filter of index_mma.cu."""
@@ -72,6 +82,8 @@ def kernels_per_step(wl):
     several rows per sequence 6 on the tensor-core path (prep, sampled pass, threshold, filter, final
     selection, and the exact scan, which returns at once when no row was handed back), else 1;
     attention 1."""
+    if wl.mode == "latent":
+        return 1
     if wl.mode == "minimal":
         return 2
     if wl.mode in ("full", "reindex"):
@@ -98,6 +110,17 @@ def fp4_tensor_peak():
         if "bf16_tflops" in d:
             return 4.0 * float(d["bf16_tflops"]), "measured bf16 burst x 4"
     return 4.0 * 1590.0, "fallback bf16 1.59 PFLOP/s x 4"
+
+
+def bf16_peak():
+    """Dense bf16 (= fp16) tensor TFLOP/s: the measured cuBLAS burst figure, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured bf16 burst"
+    return 1590.0, "fallback bf16 1.59 PFLOP/s"
 
 
 def kernel_source_hash(name):
@@ -489,6 +512,9 @@ def run_gpu(args):
     launches = args.steps * kernels_per_step(wl)
     if wl.mode == "minimal":
         kms.pop("index", None)
+    if wl.mode == "latent":
+        kms.pop("index", None)
+        kms.pop("append", None)
 
     # ---- end to end: host inputs -> C ABI call -> host outputs ----
     e2e = run_e2e(step, args, world, barrier)
@@ -510,7 +536,16 @@ def run_gpu(args):
     for k, t_ms in kms.items():
         if t_ms <= 0:
             continue
-        if wl.mode == "prefill" and k == "index":
+        if wl.mode == "latent":
+            # both contractions (S^T = L Q^T and O^T = L^T P^T) on fp16 tensor cores, next to the bytes
+            nbytes = ab[k] * B
+            flops = latent_flops(wl) * B
+            per_kernel[k] = {"algorithmic_bytes_per_launch": int(nbytes), "ms_per_launch": round(t_ms, 5),
+                             "achieved_gbs": round(nbytes / (t_ms / 1e3) / 1e9, 1),
+                             "frac": round(nbytes / (t_ms / 1e3) / 1e9 / peak, 4),
+                             "flops_per_launch": flops, "achieved_tflops": round(flops / (t_ms / 1e3) / 1e12, 1),
+                             "tensor_frac_of_bf16_peak": round(flops / (t_ms / 1e3) / 1e12 / bf16_peak()[0], 4)}
+        elif wl.mode == "prefill" and k == "index":
             tf = 2.0 * macs / (t_ms / 1e3) / 1e12
             per_kernel[k] = {"bound": "tensor", "flops_per_launch": 2.0 * macs, "ms_per_launch": round(t_ms, 5),
                              "achieved_tflops": round(tf, 1), "frac": round(tf / tpeak, 4)}
@@ -519,7 +554,7 @@ def run_gpu(args):
             per_kernel[k] = {"algorithmic_bytes_per_launch": int(round(nbytes)), "ms_per_launch": round(t_ms, 5),
                              "achieved_gbs": round(nbytes / (t_ms / 1e3) / 1e9, 1),
                              "frac": round(nbytes / (t_ms / 1e3) / 1e9 / peak, 4)}
-    dom = "attend" if wl.mode == "minimal" else "index"
+    dom = "attend" if wl.mode in ("minimal", "latent") else "index"
     mma_kernels = ("mma_prep_kernel + mma_score_kernel (sampled pass) + mma_tau_kernel + mma_score_kernel "
                    "(tensor-core filter) + mma_final_kernel + index_kernel (rows handed back)")
     if wl.mode == "prefill":
@@ -533,6 +568,8 @@ def run_gpu(args):
         # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
         if dom == "index":
             dom_file, dom_kernels = "index_decode.cu", "zero_kernel + score_kernel + select_kernel"
+        elif wl.mode == "latent":
+            dom_file, dom_kernels = "latent.cu", "latent_attend_kernel"
         else:
             dom_file, dom_kernels = "attend.cu", "attend_kernel"
     dur_s = kms[dom] / 1e3
@@ -559,8 +596,11 @@ def run_gpu(args):
                 "of the workload statement never engages)",
         "config": {"workload": args.workload + (f"@ctx{wl.context}" if args.context else ""), "mode": wl.mode,
                    "batch_per_gpu": B, "query_rows_per_sequence": wl.tq, "context": wl.context,
-                   "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": 16, "head_dim": 128,
-                   "indexer": "4 heads x 64, FP4", "kv_cache": "E2M1 + E4M3/16 (FP4), window FP8",
+                   "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": wl.hq, "head_dim": wl.d,
+                   "indexer": ("none in the step (inherited selection)" if wl.mode == "latent" else
+                               "4 heads x 64, FP4"),
+                   "kv_cache": ("one 512-channel latent per entry (K = V), E2M1 + E4M3/16, window FP8 x 512"
+                                if wl.mode == "latent" else "E2M1 + E4M3/16 (FP4), window FP8"),
                    "window": wl.win, "parallelism": f"dp{world}",
                    "l2": (f"L2 flushed between timed steps (a step reads {step_bytes / 1e6:.0f} MB, less than the L2)"
                           if flush else f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB read per step)"),
@@ -686,6 +726,8 @@ def run_e2e(step, args, world, barrier):
 
 def e2e_call(mode):
     """The public entry point(s) one end-to-end step goes through."""
+    if mode == "latent":
+        return "csa2_latent_attend"
     if mode == "prefill":
         return "csa2_prefill_chunk"
     if mode == "draft":

@@ -49,6 +49,7 @@ EXPORTS = (
     "csa2_quantize_append", "csa2_index_topk_full", "csa2_index_topk_reindex", "csa2_sparse_attend",
     "csa2_decode_full", "csa2_decode_reindex", "csa2_decode_minimal", "csa2_prefill_chunk",
     "csa2_get_device_status", "csa2_sparse_attend_noalloc", "csa2_mx_entry_bytes", "csa2_mxfp4_quantize",
+    "csa2_latent_append", "csa2_latent_attend",
 )
 
 
@@ -70,6 +71,14 @@ class csa2_cache(ctypes.Structure):
     ]
 
 
+class csa2_latent_cache(ctypes.Structure):
+    _fields_ = [
+        ("l_data", ctypes.c_void_p), ("l_scale", ctypes.c_void_p), ("k_data", ctypes.c_void_p),
+        ("k_scale", ctypes.c_void_p), ("swa", ctypes.c_void_p), ("cap", ctypes.c_int64),
+        ("swa_cap", ctypes.c_int64),
+    ]
+
+
 _lib = None
 
 
@@ -82,6 +91,7 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         vp, i, i64, u32, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t
         S, C = ctypes.POINTER(csa2_shape), ctypes.POINTER(csa2_cache)
+        LC = ctypes.POINTER(csa2_latent_cache)
         sig = {
             "csa2_entry_bytes": (sz, [i]),
             "csa2_status_string": (ctypes.c_char_p, [i]),
@@ -100,6 +110,8 @@ def lib():
             "csa2_sparse_attend_noalloc": (i, [S, C, i, i, vp, vp, vp, i, vp, f, vp, vp, vp, vp]),
             "csa2_mx_entry_bytes": (sz, [i]),
             "csa2_mxfp4_quantize": (i, [vp, i64, i, vp, vp, vp]),
+            "csa2_latent_append": (i, [LC, i, i, vp, vp, vp, vp, vp, sz, vp]),
+            "csa2_latent_attend": (i, [LC, i, i, vp, vp, vp, i, vp, i, i, f, vp, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -189,6 +201,43 @@ class Cache:
     @property
     def ref(self):
         return ctypes.byref(self.c)
+
+
+class LatentCache:
+    """Cache planes of the pages' own shape (include/csa2.h, csa2_latent_cache) for `batch`
+    sequences: the 512-channel latent (E2M1 + E4M3 per 16), the 128-channel MXFP4 indexer key and
+    a ring of 512-channel E4M3 window rows, allocated with torch."""
+
+    def __init__(self, batch: int, cap: int, swa_cap: int = 128, device="cuda", indexer=True):
+        assert swa_cap & (swa_cap - 1) == 0
+        self.batch, self.cap, self.swa_cap = batch, cap, swa_cap
+        z = lambda *s: torch.zeros(*s, dtype=torch.uint8, device=device)
+        self.l_data = z(batch, cap, 256)
+        self.l_scale = z(batch, cap, 32)
+        self.k_data = z(batch, cap, 64) if indexer else None
+        self.k_scale = z(batch, cap, 4) if indexer else None
+        self.swa = z(batch, swa_cap, 512)
+        self.c = csa2_latent_cache(_p(self.l_data), _p(self.l_scale), _p(self.k_data), _p(self.k_scale),
+                                   _p(self.swa), cap, swa_cap)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def csa2_latent_append(cache: LatentCache, batch, t, pos, latent=None, idx_k=None, swa=None, ws=None, stream=None):
+    """latent [B, t, 512], idx_k [B, t, 128], swa [B, t, 512] bf16 (any may be None) at pos [B] int64."""
+    _check("csa2_latent_append", lib().csa2_latent_append(
+        cache.ref, batch, t, _i64(pos), _bits(latent), _bits(idx_k), _bits(swa), ws.ptr if ws else None,
+        ws.nbytes if ws else 0, _stream(stream)))
+
+
+def csa2_latent_attend(cache: LatentCache, batch, tq, qpos, q, idx, k, out, swa_begin=None, win=128, ratio=1,
+                       sm_scale=0.0, out_f32=None, lse=None, ws=None, stream=None):
+    """q [B*tq, 64, 512] bf16, idx [B*tq, k] int32 -> out [B*tq, 64, 512] bf16 (tensor cores)."""
+    _check("csa2_latent_attend", lib().csa2_latent_attend(
+        cache.ref, batch, tq, _i64(qpos), _bits(q), _i32(idx), k, _i64(swa_begin), win, ratio, sm_scale, _bits(out),
+        _f32(out_f32), _f32(lse), ws.ptr if ws else None, ws.nbytes if ws else 0, _stream(stream)))
 
 
 def csa2_entry_bytes(channels: int) -> int:

@@ -1,7 +1,7 @@
 // abi.cu -- the extern "C" entry points of libcsa2 (declared and documented in include/csa2.h):
 // argument validation, workspace planning, kernel launches, status codes. Nothing here computes
-// any part of the layer step; every step runs in the kernels of append.cu, index.cu, index_decode.cu
-// and attend.cu.
+// any part of the layer step; every step runs in the kernels of append.cu, index.cu, index_decode.cu,
+// index_mma.cu, attend.cu, noalloc.cu and latent.cu.
 #include <math.h>
 
 #include "csa2_internal.cuh"
@@ -179,6 +179,67 @@ csa2_status csa2_mxfp4_quantize(const uint16_t* x, int64_t rows, int channels, u
         return CSA2_ERR_INVALID_ARG;
     if (rows == 0) return CSA2_OK;
     return from_cuda(launch_mxfp4(x, (long long)rows, channels, data, scale, (cudaStream_t)stream));
+}
+
+csa2_status csa2_latent_append(const csa2_latent_cache* cache, int batch, int t, const int64_t* pos,
+                               const uint16_t* latent, const uint16_t* idx_k, const uint16_t* swa, void* ws,
+                               size_t ws_bytes, void* stream) {
+    if (!cache || !pos || batch < 0 || t < 0) return CSA2_ERR_INVALID_ARG;
+    if (cache->cap <= 0 || cache->swa_cap <= 0 || (cache->swa_cap & (cache->swa_cap - 1))) return CSA2_ERR_INVALID_ARG;
+    if (cache->cap > ((int64_t)1 << 30)) return CSA2_ERR_CAPACITY;
+    if (latent && (!al16(latent) || !cache->l_data || !cache->l_scale || !al16(cache->l_data) || !al16(cache->l_scale)))
+        return CSA2_ERR_INVALID_ARG;
+    if (idx_k && (!al16(idx_k) || !cache->k_data || !cache->k_scale || !al16(cache->k_data) || !al16(cache->k_scale)))
+        return CSA2_ERR_INVALID_ARG;
+    if (swa && (!al16(swa) || !cache->swa || !al16(cache->swa))) return CSA2_ERR_INVALID_ARG;
+    if (ws && ws_bytes < 256) return CSA2_ERR_WORKSPACE;
+    if (batch == 0 || t == 0 || (!latent && !idx_k && !swa)) return CSA2_OK;
+    if ((latent || idx_k) && t > cache->cap) return CSA2_ERR_CAPACITY;
+    LatentAppendArgs a{};
+    a.c = *cache;
+    a.batch = batch;
+    a.t = t;
+    a.pos = pos;
+    a.latent = latent;
+    a.idx_k = idx_k;
+    a.swa = swa;
+    a.status = ws ? reinterpret_cast<uint32_t*>(ws) : nullptr;
+    return from_cuda(launch_latent_append(a, (cudaStream_t)stream));
+}
+
+csa2_status csa2_latent_attend(const csa2_latent_cache* cache, int batch, int tq, const int64_t* qpos,
+                               const uint16_t* q, const int32_t* idx, int k, const int64_t* swa_begin, int win,
+                               int ratio, float sm_scale, uint16_t* out, float* out_f32, float* lse, void* ws,
+                               size_t ws_bytes, void* stream) {
+    if (!cache || !qpos || !q || !out || batch < 0 || tq < 1 || k < 0 || k > kMaxK) return CSA2_ERR_INVALID_ARG;
+    if (win < 0 || win > 128 || (ratio != 1 && ratio != 2)) return CSA2_ERR_UNSUPPORTED_SHAPE;
+    if (cache->cap <= 0 || cache->swa_cap <= 0 || (cache->swa_cap & (cache->swa_cap - 1))) return CSA2_ERR_INVALID_ARG;
+    if (cache->cap > ((int64_t)1 << 30)) return CSA2_ERR_CAPACITY;
+    if (win > 0 && cache->swa_cap < win) return CSA2_ERR_CAPACITY;  // the ring must hold the window
+    if (k > 0 && (!idx || !cache->l_data || !cache->l_scale || !al16(cache->l_data) || !al16(cache->l_scale)))
+        return CSA2_ERR_INVALID_ARG;
+    if (win > 0 && (!cache->swa || !al16(cache->swa))) return CSA2_ERR_INVALID_ARG;
+    if (!al16(q) || !al16(out) || (out_f32 && !al16(out_f32))) return CSA2_ERR_INVALID_ARG;
+    if (ws && ws_bytes < 256) return CSA2_ERR_WORKSPACE;
+    if ((long long)batch * tq > (1ll << 31) - 1) return CSA2_ERR_INVALID_ARG;
+    if (batch == 0) return CSA2_OK;
+    LatentAttendArgs a{};
+    a.c = *cache;
+    a.rows = batch * tq;
+    a.tq = tq;
+    a.k = k;
+    a.win = win;
+    a.ratio = ratio;
+    a.qpos = qpos;
+    a.swa_begin = swa_begin;
+    a.q = q;
+    a.idx = idx;
+    a.sm_scale = sm_scale == 0.f ? 1.0f / sqrtf((float)kLatD) : sm_scale;
+    a.out = out;
+    a.out_f32 = out_f32;
+    a.lse = lse;
+    a.status = ws ? reinterpret_cast<uint32_t*>(ws) : nullptr;
+    return from_cuda(launch_latent_attend(a, (cudaStream_t)stream));
 }
 
 const char* csa2_status_string(csa2_status s) {

@@ -482,4 +482,40 @@ struct AttendArgs {
 };
 cudaError_t launch_attend(const AttendArgs& a, cudaStream_t s);
 
+// ---- the pages' own shape: the 512-channel latent (append.cu, latent.cu) ----------------------------
+constexpr int kLatD = 512;       // latent channels (K = V)
+constexpr int kLatHQ = 64;       // query heads
+constexpr int kLatBytes = 256;   // E2M1 bytes of one latent entry
+constexpr int kLatScales = 32;   // E4M3 scale bytes of one latent entry
+constexpr int kLatKBytes = 64;   // MXFP4 codes of the 128-channel indexer key
+constexpr int kLatKScales = 4;   // its E8M0 scales
+constexpr int kLatSwa = 512;     // E4M3 bytes of one window row
+
+struct LatentAppendArgs {
+    csa2_latent_cache c;
+    int batch, t;
+    const int64_t* pos;  // [batch]
+    const uint16_t* latent;
+    const uint16_t* idx_k;
+    const uint16_t* swa;
+    uint32_t* status;
+};
+cudaError_t launch_latent_append(const LatentAppendArgs& a, cudaStream_t s);
+
+struct LatentAttendArgs {
+    csa2_latent_cache c;
+    int rows, tq, k, win, ratio;
+    const int64_t* qpos;       // [rows]
+    const int64_t* swa_begin;  // [rows / tq] or NULL
+    const uint16_t* q;
+    const int32_t* idx;
+    float sm_scale;
+    uint16_t* out;
+    float* out_f32;
+    float* lse;
+    uint32_t* status;
+};
+size_t latent_attend_smem_bytes();
+cudaError_t launch_latent_attend(const LatentAttendArgs& a, cudaStream_t s);
+
 }  // namespace csa2

@@ -1,0 +1,413 @@
+// latent.cu -- sparse attention in the pages' own shape on the tensor cores: 64 query heads of 512
+// channels over a 512-channel latent that is both key and value.
+//
+// [C] "DeepSeek-V4.1-Flash: Pushing KV Cache Compression to 890 Bytes per Token":
+//   sec. VII: the main KV is one 512-channel latent per entry (288 B: E2M1 codes and an E4M3 scale
+//   per 16 channels); the configuration list: 64 query heads of dimension 512;
+//   sec. VI: the query attends to its selected entries plus its own recent window;
+//   sec. XI: cached values are dequantised before attention (E2M1 x E4M3 products and E4M3 window
+//   values are exact in fp16);
+//   sec. XII: a query at token i sees window tokens [max(s, i - win + 1), i].
+// Reading taken here: one softmax over selected and window entries, the latent serving as K and
+// V (no separate value projection), default scale 1/sqrt(512).
+//
+// One CTA per query row, 16 warps. The row's keys come in tiles of 128: ceil(k / 128) tiles of
+// selected entries (-1 or invalid entries are zero rows, masked), then one tile of up to 128 window
+// rows. Per tile:
+//   1. the tile's raw rows (loaded into registers while the previous tile was being processed) are
+//      dequantised ONCE into a 128 x 512 fp16 tile L in shared memory (K-major rows of 128-byte
+//      swizzled 64-channel blocks);
+//   2. S^T = L Q^T on tcgen05 (kind::f16, M = 128 keys, N = 64 heads, K = 512), fp32 in tensor
+//      memory;
+//   3. softmax: each thread holds one key's logits for 16 heads; the tile's per-head maxima are
+//      reduced across the CTA; the running maximum m of a head moves only when the tile exceeds it
+//      by more than 8 (in log2 units), and then the head's accumulated O and l are rescaled (in
+//      tensor memory), so P = exp2(logit - m) <= 2^8 stays well inside fp16; P is rounded to fp16
+//      into shared memory, [key][head] (MN-major);
+//   4. O^T += L^T P^T on tcgen05 (M = 128 channels, four M tiles, N = 64 heads, K = 128 keys): the
+//      same shared-memory bytes of L, read MN-major (channels contiguous), so the latent is
+//      dequantised once for both products.
+// Tensor memory: S^T in columns 0..63, O^T in columns 64..319 (channels on the lanes).
+// The result is normalised by the per-head sum of P at the end: out = O / l, lse = m ln 2 + ln l.
+// Every wait on the tensor cores is bounded; one that runs out sets CSA2_DEV_TIMEOUT.
+#include "csa2_internal.cuh"
+#include "tc.cuh"
+
+namespace csa2 {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kT = 512;                       // threads: key = tid & 127, channels 128 (tid >> 7) .. +127
+constexpr int kTile = 128;                    // keys per tile (MMA M of S^T)
+constexpr int kBlk = kTile * 128;             // 16384: one 64-channel block of the L tile
+constexpr int kLTile = 8 * kBlk;              // 131072: the fp16 L tile
+constexpr int kQBlk = kLatHQ * 128;           // 8192: one 64-channel block of Q (64 heads)
+constexpr int kQBytes = 8 * kQBlk;            // 65536
+constexpr int kPBytes = kTile * 128;          // 16384: P, 128 keys x 64 heads fp16
+constexpr uint32_t kCols = 512;               // tensor memory allocated (power of two >= 320)
+constexpr uint32_t kSCol = 0, kOCol = 64;
+constexpr float kLazy = 8.f;
+constexpr uint64_t kWaitNs = 200000000ull;
+// f16 x f16 -> f32, M 128, N 64; S^T: both operands K-major; O^T: both MN-major (bits 15, 16)
+constexpr uint32_t kIdescS = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescO = kIdescS | (1u << 15) | (1u << 16);
+constexpr size_t kOffQ = kLTile, kOffP = kOffQ + kQBytes, kOffRed = kOffP + kPBytes;
+constexpr size_t kOffM = kOffRed + 4 * 64 * 4, kOffAl = kOffM + 64 * 4, kOffL = kOffAl + 64 * 4;
+constexpr size_t kOffBar = kOffL + 64 * 4, kOffSlot = kOffBar + 16;
+constexpr size_t kUsed = kOffSlot + 16;
+// the whole 227 KB: one CTA per SM (tensor memory and the L tile allow no second one)
+constexpr size_t kSmem = 232448;
+static_assert(kUsed + 1024 <= kSmem, "shared memory plan");
+
+__device__ __forceinline__ void mma_f16(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d), "l"(ad), "l"(bd), "r"(idesc), "r"((uint32_t)acc)
+        : "memory");
+}
+
+// MN-major operand in the 128-byte swizzle pattern: 64-element groups of the M (or N) dimension
+// `lbo` bytes apart, 8-row groups of K 1024 bytes apart.
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t addr, uint32_t lbo) {
+    return sw128_desc(addr) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16);
+}
+
+// byte offset of 16-byte chunk c of row r in a 128-byte-swizzled block (8-row groups of 1024 bytes)
+__device__ __forceinline__ uint32_t sw(int r, int c) { return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)); }
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t scale_h2(uint32_t s) { return e4m3x2_to_h2((uint16_t)(s | (s << 8))); }
+
+// 16 lanes' worth of values reduced across the warp: lane L < 16 ends with op over all 32 lanes of
+// element L (the transposing butterfly: each step halves the elements a lane keeps).
+template <bool kMax>
+__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, v[i], 16);
+        v[i] = kMax ? fmaxf(v[i], o) : v[i] + o;
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1) {
+        const bool up = (lane & w) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float keep = up ? v[i + w] : v[i], send = up ? v[i] : v[i + w];
+            const float o = __shfl_xor_sync(0xffffffffu, send, w);
+            v[i] = kMax ? fmaxf(keep, o) : keep + o;
+        }
+    }
+    return v[0];
+}
+
+__global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    unsigned char* Lt = sm;
+    unsigned char* Qs = sm + kOffQ;
+    unsigned char* Ps = sm + kOffP;
+    float* red = reinterpret_cast<float*>(sm + kOffRed);   // [4 lane quarters][64 heads]
+    float* s_m = reinterpret_cast<float*>(sm + kOffM);     // running maximum per head (log2 units)
+    float* s_al = reinterpret_cast<float*>(sm + kOffAl);   // this tile's rescale factor per head
+    float* s_l = reinterpret_cast<float*>(sm + kOffL);     // final sum per head
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [0] S^T done, [1] O^T done
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kOffSlot);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int key = tid & 127, qq = tid >> 7;      // load / dequantise: key, channels 128 qq ..
+    const int quad = warp & 3, cg = warp >> 2;     // softmax / epilogue: lanes 32 quad .., heads 16 cg ..
+    const int row = blockIdx.x, K = a.k;
+    wait_prior_grid();  // indices, cache and queries come from earlier work on the stream
+
+    const int b = row / a.tq;
+    const int64_t qpos = a.qpos[row];
+    const int64_t qlast = qpos < 0 ? -1 : (qpos + 1) / a.ratio - 1;  // the last visible entry
+    const bool row_ok = qpos >= 0 && qlast < a.c.cap;
+    int64_t lo = qpos - a.win + 1;
+    {
+        const int64_t sb = a.swa_begin ? a.swa_begin[b] : 0;
+        if (lo < sb) lo = sb;
+        if (lo < 0) lo = 0;
+    }
+    const int nwin = (row_ok && qpos >= lo) ? (int)(qpos - lo + 1) : 0;
+    const int ft = row_ok ? (K + kTile - 1) / kTile : 0;
+    const int nt = ft + (nwin > 0 ? 1 : 0);
+    const float scale2 = a.sm_scale * 1.4426950408889634f;  // logits in log2 units
+
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        mbar_fence_init();
+    }
+    if (tid < 64) s_m[tid] = -INFINITY;
+    if (warp == 0) tmem_alloc(tslot, kCols);
+    {   // Q -> fp16 (B operand of S^T, K-major): thread -> head tid >> 3, channels 64 (tid & 7) ..
+        const int h = tid >> 3, cb = tid & 7;
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)row * kLatHQ + h) * kLatD + 64 * cb);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint4 x = __ldg(src + c);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint32_t hv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hv[i] = pack_h2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+            *reinterpret_cast<uint4*>(Qs + cb * kQBlk + sw(h, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+    }
+
+    const size_t seq_row0 = (size_t)b * a.c.cap;
+    const size_t swa_row0 = (size_t)b * a.c.swa_cap;
+    uint32_t* status = a.status;
+    bool ok_all = true;
+    auto wait_bar = [&](int i, uint32_t parity) {
+        if (!mbar_wait(&bars[i], parity, kWaitNs)) {
+            if (ok_all) set_status(status, CSA2_DEV_TIMEOUT);
+            ok_all = false;
+        }
+    };
+
+    // ---- raw rows of tile j into registers (this thread: key `key`, channels 128 qq .. +127) ----
+    uint4 raw[8];
+    uint2 rsc;
+    bool kvalid = false;  // the key of this thread in the tile being loaded
+    auto load_tile = [&](int j) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) raw[i] = make_uint4(0, 0, 0, 0);
+        rsc = make_uint2(0, 0);
+        kvalid = false;
+        if (j < ft) {
+            const int i = j * kTile + key;
+            if (i < K) {
+                const int v = __ldg(a.idx + (size_t)row * K + i);
+                const bool ok = v >= 0 && (int64_t)v <= qlast && (int64_t)v < a.c.cap;
+                if (!ok && v != -1 && qq == 0) set_status(status, CSA2_DEV_BAD_INDEX);
+                if (ok) {
+                    kvalid = true;
+                    const uint4* src = reinterpret_cast<const uint4*>(a.c.l_data + (seq_row0 + (size_t)v) * kLatBytes + 64 * qq);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
+                    rsc = __ldg(reinterpret_cast<const uint2*>(a.c.l_scale + (seq_row0 + (size_t)v) * kLatScales + 8 * qq));
+                }
+            }
+        } else if (j < nt && key < nwin) {
+            kvalid = true;
+            const int64_t p = lo + key;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                a.c.swa + (swa_row0 + (size_t)(p & (a.c.swa_cap - 1))) * kLatSwa + 128 * qq);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) raw[c] = __ldg(src + c);
+        }
+    };
+    // dequantise the registers into the L tile: channel 128 qq + 8 c lands in 64-channel block
+    // 2 qq + c / 8, chunk c % 8, of row `key`
+    auto dequant = [&](bool fp4) {
+        if (fp4) {
+#pragma unroll
+            for (int bk = 0; bk < 8; ++bk) {  // 16-channel scale block bk: code words 2 bk, 2 bk + 1
+                const uint32_t s2 = scale_h2(((bk < 4 ? rsc.x : rsc.y) >> (8 * (bk & 3))) & 0xFFu);
+                const uint4 rw = raw[bk >> 1];
+                const uint32_t w0 = (bk & 1) ? rw.z : rw.x, w1 = (bk & 1) ? rw.w : rw.y;
+                uint32_t h0[4], h1[4];
+                e2m1x8_to_h2x4(w0, h0);
+                e2m1x8_to_h2x4(w1, h1);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { h0[i] = hmul2(h0[i], s2); h1[i] = hmul2(h1[i], s2); }
+                const int c0 = 2 * bk;  // chunk index among the thread's 16 chunks of 8 channels
+                *reinterpret_cast<uint4*>(Lt + (2 * qq + (c0 >> 3)) * kBlk + sw(key, c0 & 7)) = make_uint4(h0[0], h0[1], h0[2], h0[3]);
+                *reinterpret_cast<uint4*>(Lt + (2 * qq + ((c0 + 1) >> 3)) * kBlk + sw(key, (c0 + 1) & 7)) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {  // 8 window channels per chunk
+                const uint4 rw = raw[c >> 1];
+                const uint32_t w0 = (c & 1) ? rw.z : rw.x, w1 = (c & 1) ? rw.w : rw.y;
+                const uint4 h = make_uint4(e4m3x2_to_h2((uint16_t)(w0 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w0 >> 16)),
+                                           e4m3x2_to_h2((uint16_t)(w1 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w1 >> 16)));
+                *reinterpret_cast<uint4*>(Lt + (2 * qq + (c >> 3)) * kBlk + sw(key, c & 7)) = h;
+            }
+        }
+    };
+
+    load_tile(0);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();  // barriers, s_m, Q, tensor memory address
+    tc_fence_after();
+    const uint32_t tb = *tslot;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+
+    float lsum[16];  // this thread's key slot: sum of P per head 16 cg + i over the tiles so far
+#pragma unroll
+    for (int i = 0; i < 16; ++i) lsum[i] = 0.f;
+
+    for (int j = 0; j < nt; ++j) {
+        const bool fp4 = j < ft;  // CTA-uniform
+        const bool valid = kvalid;
+        if (j > 0) wait_bar(1, (uint32_t)(j - 1) & 1u);  // O^T of tile j - 1 has read L and P
+        dequant(fp4);
+        if (j + 1 < nt) load_tile(j + 1);  // in flight during this tile's MMAs and softmax
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < 32; ++kk) {
+                const uint32_t off = (uint32_t)((kk >> 2) * kBlk + 32 * (kk & 3));
+                const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + 32 * (kk & 3));
+                mma_f16(tb + kSCol, sw128_desc(smem_u32(Lt) + off), sw128_desc(smem_u32(Qs) + qoff), kIdescS, kk > 0);
+            }
+            mma_commit(&bars[0]);
+        }
+        wait_bar(0, (uint32_t)j & 1u);
+        tc_fence_after();
+
+        // ---- softmax of the tile: this thread's key 32 quad + lane (= key), heads 16 cg .. +15 ----
+        // (the logits are read from tensor memory twice: for the maxima, then for P, which keeps
+        // them out of registers during the reduction)
+        const uint32_t s_addr = tb + lane_base + kSCol + 16 * cg;
+        {
+            uint32_t v[16];
+            tmem_ld16(s_addr, v);
+            tmem_ld_wait();
+            float mx[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) mx[i] = valid ? __uint_as_float(v[i]) * scale2 : -INFINITY;
+            const float r = warp_reduce16<true>(mx, lane);
+            if (lane < 16) red[quad * 64 + 16 * cg + lane] = r;
+        }
+        __syncthreads();
+        int resc = 0;
+        if (tid < 64) {
+            const float tmax = fmaxf(fmaxf(red[tid], red[64 + tid]), fmaxf(red[128 + tid], red[192 + tid]));
+            const float m_old = s_m[tid];
+            float al = 1.f;
+            if (tmax > m_old + kLazy) {  // also the first finite maximum (m_old = -inf)
+                al = (m_old == -INFINITY) ? 0.f : exp2f(m_old - tmax);
+                resc = m_old != -INFINITY;
+                s_m[tid] = tmax;
+            }
+            s_al[tid] = al;
+        }
+        resc = __syncthreads_or(resc);
+        const float* al = s_al + 16 * cg;  // this warp's heads (shared-memory broadcasts)
+        const float* mh = s_m + 16 * cg;
+        if (resc) {
+            // O^T (columns = heads) of tile j - 1 is complete: scale this warp's heads in place
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                uint32_t v[16];
+                const uint32_t addr = tb + lane_base + kOCol + 64 * mt + 16 * cg;
+                tmem_ld16(addr, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * al[i]);
+                tmem_st16(addr, v);
+            }
+            tmem_st_wait();
+        }
+        uint32_t ph[8];
+        float lg[16];
+        {
+            uint32_t v[16];
+            tmem_ld16(s_addr, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) lg[i] = valid ? __uint_as_float(v[i]) * scale2 : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+            const float m0 = mh[i], m1 = mh[i + 1];
+            const float p0 = (m0 == -INFINITY) ? 0.f : exp2f(lg[i] - m0);
+            const float p1 = (m1 == -INFINITY) ? 0.f : exp2f(lg[i + 1] - m1);
+            lsum[i] = lsum[i] * al[i] + p0;
+            lsum[i + 1] = lsum[i + 1] * al[i + 1] + p1;
+            ph[i >> 1] = pack_h2(p0, p1);
+        }
+        // P [key][head]: heads 16 cg .. +7 -> chunk 2 cg, 16 cg + 8 .. -> chunk 2 cg + 1
+        *reinterpret_cast<uint4*>(Ps + sw(key, 2 * cg)) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+        *reinterpret_cast<uint4*>(Ps + sw(key, 2 * cg + 1)) = make_uint4(ph[4], ph[5], ph[6], ph[7]);
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // A = L^T: channels 128 mt .. (blocks 2 mt, 2 mt + 1, kBlk apart), keys 16 kk ..
+                    const uint64_t ad = sw128_desc_mn(smem_u32(Lt) + (uint32_t)(2 * mt * kBlk + 2048 * kk), kBlk);
+                    // B = P: heads 0..63 (one 64-element group), keys 16 kk ..
+                    const uint64_t bd = sw128_desc_mn(smem_u32(Ps) + (uint32_t)(2048 * kk), 0);
+                    mma_f16(tb + kOCol + 64 * mt, ad, bd, kIdescO, j > 0 || kk > 0);
+                }
+            }
+            mma_commit(&bars[1]);
+        }
+    }
+    if (nt > 0) {
+        wait_bar(1, (uint32_t)(nt - 1) & 1u);
+        tc_fence_after();
+    }
+
+    // ---- epilogue: l per head, then out = O / l (warp: channels 128 mt + 32 quad + lane, heads 16 cg ..) ----
+    {
+        const float r = warp_reduce16<false>(lsum, lane);
+        if (lane < 16) red[quad * 64 + 16 * cg + lane] = r;
+    }
+    __syncthreads();
+    if (tid < 64) s_l[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
+    __syncthreads();
+    float inv[16];
+    bool empty[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int h = 16 * cg + i;
+        empty[i] = (nt == 0) || (s_m[h] == -INFINITY) || !(s_l[h] > 0.f);
+        inv[i] = empty[i] ? 0.f : 1.f / s_l[h];
+    }
+#pragma unroll
+    for (int mt = 0; mt < 4; ++mt) {
+        uint32_t v[16] = {};
+        if (nt > 0) {
+            tmem_ld16(tb + lane_base + kOCol + 64 * mt + 16 * cg, v);
+            tmem_ld_wait();
+        }
+        const int d = 128 * mt + 32 * quad + lane;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float x = empty[i] ? 0.f : __uint_as_float(v[i]) * inv[i];
+            const size_t ob = ((size_t)row * kLatHQ + 16 * cg + i) * kLatD + d;
+            a.out[ob] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+            if (a.out_f32) a.out_f32[ob] = x;
+        }
+    }
+    if (a.lse && tid < 64) {
+        const bool e = (nt == 0) || (s_m[tid] == -INFINITY) || !(s_l[tid] > 0.f);
+        a.lse[(size_t)row * kLatHQ + tid] = e ? -INFINITY : (s_m[tid] * 0.6931471805599453f + logf(s_l[tid]));
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tb, kCols);
+}
+
+}  // namespace
+
+size_t latent_attend_smem_bytes() { return kSmem; }
+
+cudaError_t launch_latent_attend(const LatentAttendArgs& a, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(latent_attend_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
+    if (a.rows == 0) return cudaSuccess;
+    return launch_after_prior(latent_attend_kernel, dim3((unsigned)a.rows), dim3(kT), kSmem, s, a);
+}
+
+}  // namespace csa2

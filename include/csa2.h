@@ -293,6 +293,66 @@ CSA2_API csa2_status csa2_sparse_attend_noalloc(const csa2_shape* shape, const c
 CSA2_API csa2_status csa2_mxfp4_quantize(const uint16_t* x, int64_t rows, int channels, uint8_t* data, uint8_t* scale,
                                          void* stream);
 
+/*
+ * The pages' own attention shape ([C] sec. VII: the main KV is ONE 512-channel latent per entry,
+ * 288 B in E2M1 with an E4M3 scale per 16 channels; the configuration list of [C]'s closing
+ * section: 64 query heads of dimension 512, an indexer of 32 heads x 128 over one 128-channel
+ * MXFP4 key per entry). The latent is both K and V. Cache of `batch` sequences, per sequence b
+ * and position p (0 <= p < cap); every plane base 16-byte aligned; the caller owns every plane:
+ *   l_data  + (b*cap + p)*256     : the latent's 512 channels as E2M1 codes (channel 2j in the
+ *                                    low nibble of byte j)
+ *   l_scale + (b*cap + p)*32      : one E4M3 scale per 16 channels (the codec of this header)
+ *   k_data  + (b*cap + p)*64      : the 128-channel indexer key as MXFP4 codes
+ *   k_scale + (b*cap + p)*4       : its E8M0 scales (one per 32 channels; see csa2_mxfp4_quantize)
+ *   swa     + (b*swa_cap + (p & (swa_cap-1)))*512 : window rows, 512 E4M3 bytes, no scale
+ */
+typedef struct {
+    uint8_t* l_data;
+    uint8_t* l_scale;
+    uint8_t* k_data;
+    uint8_t* k_scale;
+    uint8_t* swa;
+    int64_t cap;      /* positions per sequence (<= 2^30) */
+    int64_t swa_cap;  /* ring slots per sequence, power of two */
+} csa2_latent_cache;
+
+/*
+ * Quantise-append of t tokens per sequence into the latent cache, at positions pos[b] .. pos[b]
+ * + t - 1 ([C] sec. XI: quantised as they are written; the window stays FP8):
+ *   latent [batch][t][512], idx_k [batch][t][128], swa [batch][t][512] (bf16, 16-byte aligned;
+ *   any may be NULL, and its plane is then neither read nor written). The latent takes the
+ *   E2M1/E4M3 codec of csa2_quantize_append, the key the MXFP4 rule of csa2_mxfp4_quantize,
+ *   window rows E4M3 (RNE, saturating). A position outside [0, cap) sets CSA2_DEV_BAD_POS in
+ *   `ws` (which may be NULL: the bit is then not recorded) and that sequence is skipped.
+ * Returns CSA2_ERR_INVALID_ARG for null / misaligned pointers or negative sizes.
+ */
+CSA2_API csa2_status csa2_latent_append(const csa2_latent_cache* cache, int batch, int t, const int64_t* pos,
+                                        const uint16_t* latent, const uint16_t* idx_k, const uint16_t* swa, void* ws,
+                                        size_t ws_bytes, void* stream);
+
+/*
+ * Sparse attention of the pages' own shape, on the tensor cores: each of the batch*tq query rows
+ * (64 heads x 512 channels, bf16) attends in ONE softmax to its selected latent entries and its
+ * window rows, the latent being both key and value ([C] sec. VI, VII, XII):
+ *   qpos [batch*tq] token of each row; idx [batch*tq][k] selected entries (-1 = none), each
+ *   visible at its row ((qpos + 1) / ratio entries are); window tokens [max(swa_begin[b],
+ *   qpos - win + 1, 0), qpos] with win <= 128 (swa_begin may be NULL: 0); sm_scale 0 gives
+ *   1/sqrt(512); ratio 1 or 2 (the entry rule of csa2_shape.ratio).
+ *   out [batch*tq][64][512] bf16; out_f32 (same shape, fp32) and lse [batch*tq][64] (natural
+ *   log) may be NULL. A row with no key gives out = 0 and lse = -inf.
+ *   ws: a workspace of at least 256 bytes initialised by csa2_workspace_init (its status word
+ *   receives CSA2_DEV_BAD_INDEX for an index < -1, not visible or >= cap, which is skipped, and
+ *   CSA2_DEV_TIMEOUT if a tensor-core wait ran out); NULL leaves such bits unrecorded.
+ * Precision: q is rounded bf16 -> fp16 (exact for 2^-14 <= |q| <= 65504), the dequantised latent
+ * is exact in fp16, logits and sums are fp32, probabilities are rounded to fp16.
+ * Returns CSA2_ERR_INVALID_ARG for null / misaligned pointers, k < 0 or k > 2048, win outside
+ * 0..128 or a bad ratio.
+ */
+CSA2_API csa2_status csa2_latent_attend(const csa2_latent_cache* cache, int batch, int tq, const int64_t* qpos,
+                                        const uint16_t* q, const int32_t* idx, int k, const int64_t* swa_begin,
+                                        int win, int ratio, float sm_scale, uint16_t* out, float* out_f32, float* lse,
+                                        void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word in `ws`.
  * *host_status receives the CSA2_DEV_* bits; returns CSA2_ERR_DEVICE if any bit was set. */
 CSA2_API csa2_status csa2_get_device_status(void* ws, void* stream, int32_t* host_status /* host */);

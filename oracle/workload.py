@@ -10,7 +10,7 @@ import torch
 
 import workloads as W
 
-from . import SeqCache
+from . import LatentCache, SeqCache
 
 
 def _v(seed, stream, b, p, width):
@@ -26,6 +26,18 @@ def build_sequence(wl, b):
     """Returns (cache, inputs) of sequence b before its step."""
     N, seed = wl.context, wl.seed
     inp = {}
+    if wl.mode == "latent":
+        # the pages' own shape: the latent rows of the selected entries and the window rows
+        c = LatentCache(cap=N, swa_cap=128)
+        idx = W.distinct_sorted(seed, "sel", torch.tensor([b]), N - 1, wl.k)[0].numpy()
+        inp["idx"] = idx.astype(np.int32)
+        lat = _v(seed, "lat", b, idx.astype(np.int64), 512)
+        for j, pp in enumerate(idx):
+            c.append(int(pp), latent=lat[j:j + 1])
+        pw = torch.arange(N - wl.win, N)
+        c.append(N - wl.win, swa=_v(seed, "lsw", b, pw, 512))
+        inp["q"] = _v(seed, "lq", b, [N - 1], 64 * 512)[0].reshape(64, 512)
+        return c, inp
     if wl.mode == "prefill":
         p0 = N - wl.tq
         c = SeqCache(cap=N, swa_cap=1 << (wl.tq + wl.win - 1).bit_length())
@@ -89,6 +101,10 @@ def run_step(c, wl, inp, rows=None):
     rows = {row: (idx, out, lse)}."""
     N = wl.context
     r = {}
+    if wl.mode == "latent":
+        r["idx"] = inp["idx"]
+        r["out"], r["lse"] = c.attend(N - 1, inp["q"], inp["idx"], win=wl.win)
+        return r
     if wl.mode in ("prefill", "draft"):
         p0 = N - wl.tq
         c.append(p0, kv=inp["kv"], idx_k=inp["idx_k"], swa_kv=inp["swa_kv"])

@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_symbols()
-    assert len(names) == 17
+    assert len(names) == 19
     assert set(names) == set(csa.EXPORTS)
     for n in names:
         assert hasattr(L, n), n
@@ -39,7 +39,7 @@ def test_header_compiles_as_c():
     with tempfile.TemporaryDirectory() as d:
         c = os.path.join(d, "t.c")
         with open(c, "w") as f:
-            f.write('#include "csa2.h"\nint main(void){ csa2_shape s; csa2_cache c; (void)s; (void)c; return 0; }\n')
+            f.write('#include "csa2.h"\nint main(void){ csa2_shape s; csa2_cache c; csa2_latent_cache l; (void)s; (void)c; (void)l; return 0; }\n')
         subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), "-c", c,
                                "-o", os.path.join(d, "t.o")])
 
@@ -242,3 +242,39 @@ def test_mx_entry_bytes_and_codec_validation(L):
     assert f(base, -1, 32, base, base, None) == csa.CSA2_ERR_INVALID_ARG
     assert f(base + 2, 1, 32, base, base, None) == csa.CSA2_ERR_INVALID_ARG
     assert f(base, 0, 32, base, base, None) == csa.CSA2_OK  # nothing to do, no launch
+
+
+def test_latent_entry_points_validate_before_any_launch(L):
+    """The pages' own shape (latent cache, 64 x 512 attention): bad pointers, alignment, sizes, window
+    and ratio are rejected on the host; an empty batch returns OK without a launch."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    base = (ctypes.addressof(buf) + 255) & ~255
+    c = csa.csa2_latent_cache(base, base + 4096, base + 8192, base + 12288, base + 16384, 1024, 128)
+    rc = ctypes.byref(c)
+    att, app = L.csa2_latent_attend, L.csa2_latent_append
+    q = out = idx = qpos = base + 32768
+    # (cache, batch, tq, qpos, q, idx, k, swa_begin, win, ratio, sm_scale, out, out_f32, lse, ws, ws_bytes, stream)
+    assert att(rc, 0, 1, qpos, q, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_OK
+    assert att(None, 0, 1, qpos, q, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert att(rc, 0, 1, None, q, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert att(rc, 0, 1, qpos, q + 2, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert att(rc, 0, 1, qpos, q, idx, 4096, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert att(rc, 0, 1, qpos, q, None, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert att(rc, 0, 1, qpos, q, idx, 512, None, 129, 1, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    assert att(rc, 0, 1, qpos, q, idx, 512, None, 128, 3, 0.0, out, None, None, None, 0, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    assert att(rc, 0, 1, qpos, q, idx, 512, None, 128, 1, 0.0, out, None, None, base, 16, None) == csa.CSA2_ERR_WORKSPACE
+    small = csa.csa2_latent_cache(base, base + 4096, base + 8192, base + 12288, base + 16384, 1024, 64)
+    assert att(ctypes.byref(small), 0, 1, qpos, q, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == \
+        csa.CSA2_ERR_CAPACITY  # the window ring is shorter than the window
+    odd = csa.csa2_latent_cache(base + 8, base + 4096, base + 8192, base + 12288, base + 16384, 1024, 128)
+    assert att(ctypes.byref(odd), 0, 1, qpos, q, idx, 512, None, 128, 1, 0.0, out, None, None, None, 0, None) == \
+        csa.CSA2_ERR_INVALID_ARG
+    # (cache, batch, t, pos, latent, idx_k, swa, ws, ws_bytes, stream)
+    x = base + 40960
+    assert app(rc, 0, 1, qpos, x, x, x, None, 0, None) == csa.CSA2_OK
+    assert app(rc, 1, 1, None, x, x, x, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert app(rc, -1, 1, qpos, x, x, x, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert app(rc, 1, 1, qpos, x + 2, None, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+    assert app(rc, 1, 2048, qpos, x, None, None, None, 0, None) == csa.CSA2_ERR_CAPACITY
+    nokey = csa.csa2_latent_cache(base, base + 4096, None, None, base + 16384, 1024, 128)
+    assert app(ctypes.byref(nokey), 1, 1, qpos, None, x, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG

@@ -41,7 +41,9 @@ _GOLDEN = _s64(0x9E3779B97F4A7C15)
 _C1 = _s64(0xBF58476D1CE4E5B9)
 _C2 = _s64(0x94D049BB133111EB)
 
-STREAM = {"kv": 1, "ik": 2, "swa": 3, "q": 4, "iq": 5, "pool": 6, "sel": 7}
+STREAM = {"kv": 1, "ik": 2, "swa": 3, "q": 4, "iq": 5, "pool": 6, "sel": 7,
+          # the pages' own shape: 512-channel latent, 128-channel indexer key, window rows, query
+          "lat": 8, "lik": 9, "lsw": 10, "lq": 11}
 POS_BITS = 21  # positions per sequence addressed by the counters: < 2^21
 
 
@@ -113,7 +115,7 @@ def distinct_sorted(seed: int, stream, b: torch.Tensor, n_range: int, count: int
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str            # "full" | "reindex" | "minimal" | "prefill" | "draft"
+    mode: str            # "full" | "reindex" | "minimal" | "prefill" | "draft" | "latent"
     batch: int
     context: int         # N: visible positions for a decode query (query at N-1)
     seed: int
@@ -139,4 +141,7 @@ WORKLOADS = {
     # multi-token decode: each sequence appends 5 draft tokens at N-5 .. N-1 and verifies them together
     # (Full index over every visible position, row t sees positions <= N-5+t; no block pool)
     "draft_b64_n131072_tq5": Workload("draft_b64_n131072_tq5", "draft", 64, 131072, seed=5, tq=5),
+    # the pages' own attention shape: 64 query heads x 512 over the 512-channel latent (K = V), a
+    # decode row per sequence at N - 1 with 512 inherited selected entries and a 128-token window
+    "latent_b128_n131072": Workload("latent_b128_n131072", "latent", 128, 131072, seed=6, hq=64, d=512),
 }

@@ -127,6 +127,62 @@ class Step:
         hooks("attend", 1)
 
 
+class StatusWs:
+    """The 256-byte workspace csa2_latent_attend / csa2_latent_append take (its status word)."""
+
+    def __init__(self, device):
+        self.buf = torch.zeros(256, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self):
+        return self.buf.data_ptr()
+
+    @property
+    def nbytes(self):
+        return self.buf.numel()
+
+
+@dataclasses.dataclass
+class LatentStep:
+    """A decode row per sequence in the pages' own attention shape (64 heads x 512 over the
+    512-channel latent, K = V): one csa2_latent_attend call per step."""
+    wl: Workload
+    cache: csa.LatentCache
+    ws: StatusWs
+    inputs: dict
+    outputs: dict
+    batch: int
+
+    def run(self, stream=None, ws=None, out_f32=None, lse=None):
+        I, O = self.inputs, self.outputs
+        csa.csa2_latent_attend(self.cache, self.batch, 1, I["qpos"], I["q"], I["idx"], self.wl.k, O["out"],
+                               win=self.wl.win, out_f32=out_f32, lse=lse, ws=ws or self.ws, stream=stream)
+
+    def run_parts(self, hooks, stream=None):
+        hooks("attend", 0)
+        self.run(stream)
+        hooks("attend", 1)
+
+
+def _build_latent(wl, seqs, B, device):
+    N = wl.context
+    cache = csa.LatentCache(B, N, 128, device=device, indexer=False)
+    ws = StatusWs(device)
+    idx = distinct_sorted(wl.seed, "sel", seqs, N - 1, wl.k).to(torch.int32).contiguous()
+    lat = _vals(wl.seed, "lat", seqs, idx.to(torch.int64), 512)
+    for j in range(wl.k):  # the selected rows only: the step reads nothing else of the latent plane
+        csa.csa2_latent_append(cache, B, 1, idx[:, j].to(torch.int64).contiguous(), latent=lat[:, j:j + 1].contiguous(),
+                               ws=ws)
+    pw = torch.arange(N - wl.win, N, device=device)
+    csa.csa2_latent_append(cache, B, wl.win, torch.full((B,), N - wl.win, dtype=torch.int64, device=device),
+                           swa=_vals(wl.seed, "lsw", seqs, pw, 512).contiguous(), ws=ws)
+    qpos = torch.full((B,), N - 1, dtype=torch.int64, device=device)
+    q = _vals(wl.seed, "lq", seqs, qpos.unsqueeze(1), 64 * 512)[:, 0].reshape(B, 64, 512).contiguous()
+    out = torch.empty(B, 64, 512, dtype=torch.bfloat16, device=device)
+    torch.cuda.synchronize()
+    return LatentStep(wl, cache, ws, {"qpos": qpos, "q": q, "idx": idx}, {"out": out}, B)
+
+
 def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda", context=None) -> Step:
     """Allocate and fill the cache of workload `name` (optionally a smaller batch, or the sequences
     seq_offset .. seq_offset+batch-1 of it, as a data-parallel rank would; optionally another context
@@ -136,6 +192,8 @@ def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda
         wl = dataclasses.replace(wl, context=context)
     B = wl.batch if batch is None else batch
     seqs = torch.arange(seq_offset, seq_offset + B, device=device)
+    if wl.mode == "latent":
+        return _build_latent(wl, seqs, B, device)
     shape = csa.make_shape(wl.win)
     N = wl.context
     I, O = {}, {}
