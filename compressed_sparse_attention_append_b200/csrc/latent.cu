@@ -20,13 +20,19 @@
 //   2. S^T = L Q^T on tcgen05 (kind::f16, M = 128 keys, N = 64 heads, K = 512), fp32 in tensor
 //      memory;
 //   3. softmax: each thread holds one key's logits for 16 heads; the tile's per-head maxima are
-//      reduced across the CTA; the running maximum m of a head moves only when the tile exceeds it
+//      reduced across the CTA (a warp reduction per head, then the four lane quarters through
+//      shared memory); the running maximum m of a head moves only when the tile exceeds it
 //      by more than 8 (in log2 units), and then the head's accumulated O and l are rescaled (in
 //      tensor memory), so P = exp2(logit - m) <= 2^8 stays well inside fp16; P is rounded to fp16
 //      into shared memory, [key][head] (MN-major);
 //   4. O^T += L^T P^T on tcgen05 (M = 128 channels, four M tiles, N = 64 heads, K = 128 keys): the
 //      same shared-memory bytes of L, read MN-major (channels contiguous), so the latent is
 //      dequantised once for both products.
+// The two channel halves of L (64-channel blocks 0..3 and 4..7) are dequantised by separate halves
+// of the CTA, each as soon as the O^T MMAs of the previous tile that read it have completed, and the
+// S^T k-steps of a half are issued as soon as that half is in place (mbarriers between the threads
+// and the MMA issuer), so dequantisation overlaps the tensor pipe. The row's indices are checked
+// and staged in shared memory once, so no tile waits on a dependent index load.
 // Tensor memory: S^T in columns 0..63, O^T in columns 64..319 (channels on the lanes).
 // The result is normalised by the per-head sum of P at the end: out = O / l, lse = m ln 2 + ln l.
 // Every wait on the tensor cores is bounded; one that runs out sets CSA2_DEV_TIMEOUT.
@@ -53,13 +59,16 @@ constexpr uint64_t kWaitNs = 200000000ull;
 // f16 x f16 -> f32, M 128, N 64; S^T: both operands K-major; O^T: both MN-major (bits 15, 16)
 constexpr uint32_t kIdescS = (1u << 4) | ((64u >> 3) << 17) | ((128u >> 4) << 24);
 constexpr uint32_t kIdescO = kIdescS | (1u << 15) | (1u << 16);
-constexpr size_t kOffQ = kLTile, kOffP = kOffQ + kQBytes, kOffRed = kOffP + kPBytes;
+constexpr size_t kOffQ = kLTile, kOffP = kOffQ + kQBytes, kOffIdx = kOffP + kPBytes;
+constexpr size_t kOffRed = kOffIdx + 4 * kMaxK;
 constexpr size_t kOffM = kOffRed + 4 * 64 * 4, kOffAl = kOffM + 64 * 4, kOffL = kOffAl + 64 * 4;
-constexpr size_t kOffBar = kOffL + 64 * 4, kOffSlot = kOffBar + 16;
+constexpr size_t kOffBar = kOffL + 64 * 4, kOffSlot = kOffBar + 8 * 8;
 constexpr size_t kUsed = kOffSlot + 16;
 // the whole 227 KB: one CTA per SM (tensor memory and the L tile allow no second one)
 constexpr size_t kSmem = 232448;
 static_assert(kUsed + 1024 <= kSmem, "shared memory plan");
+// mbarriers: S^T done; O^T of channel half 0 / 1 done; channel half 0 / 1 of L dequantised
+enum { kBarS = 0, kBarO0 = 1, kBarO1 = 2, kBarH0 = 3, kBarH1 = 4 };
 
 __device__ __forceinline__ void mma_f16(uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, bool acc) {
     asm volatile(
@@ -84,23 +93,31 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 }
 __device__ __forceinline__ uint32_t scale_h2(uint32_t s) { return e4m3x2_to_h2((uint16_t)(s | (s << 8))); }
 
-// 16 lanes' worth of values reduced across the warp: lane L < 16 ends with op over all 32 lanes of
-// element L (the transposing butterfly: each step halves the elements a lane keeps).
-template <bool kMax>
-__device__ __forceinline__ float warp_reduce16(float (&v)[16], int lane) {
+// the largest value of v over the warp, in every lane (sm_100a warp reduction)
+__device__ __forceinline__ float warp_max(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+// 2^x (the hardware approximation: relative error about 2^-22; results below 2^-126 flush to 0)
+__device__ __forceinline__ float ex2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// 16 lanes' worth of sums reduced across the warp: lane L < 16 ends with the sum over all 32 lanes
+// of element L (the transposing butterfly: each step halves the elements a lane keeps).
+__device__ __forceinline__ float warp_sum16(float (&v)[16], int lane) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, v[i], 16);
-        v[i] = kMax ? fmaxf(v[i], o) : v[i] + o;
-    }
+    for (int i = 0; i < 16; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], 16);
 #pragma unroll
     for (int w = 8; w >= 1; w >>= 1) {
         const bool up = (lane & w) != 0;
 #pragma unroll
         for (int i = 0; i < w; ++i) {
             const float keep = up ? v[i + w] : v[i], send = up ? v[i] : v[i + w];
-            const float o = __shfl_xor_sync(0xffffffffu, send, w);
-            v[i] = kMax ? fmaxf(keep, o) : keep + o;
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
         }
     }
     return v[0];
@@ -112,15 +129,17 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
     unsigned char* Lt = sm;
     unsigned char* Qs = sm + kOffQ;
     unsigned char* Ps = sm + kOffP;
+    int* sidx = reinterpret_cast<int*>(sm + kOffIdx);       // the row's selected entries, -1 if unusable
     float* red = reinterpret_cast<float*>(sm + kOffRed);   // [4 lane quarters][64 heads]
     float* s_m = reinterpret_cast<float*>(sm + kOffM);     // running maximum per head (log2 units)
     float* s_al = reinterpret_cast<float*>(sm + kOffAl);   // this tile's rescale factor per head
     float* s_l = reinterpret_cast<float*>(sm + kOffL);     // final sum per head
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [0] S^T done, [1] O^T done
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + kOffBar);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(sm + kOffSlot);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int key = tid & 127, qq = tid >> 7;      // load / dequantise: key, channels 128 qq ..
+    const int half = qq >> 1;                      // channel half (blocks 4 half .. 4 half + 3)
     const int quad = warp & 3, cg = warp >> 2;     // softmax / epilogue: lanes 32 quad .., heads 16 cg ..
     const int row = blockIdx.x, K = a.k;
     wait_prior_grid();  // indices, cache and queries come from earlier work on the stream
@@ -139,14 +158,25 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
     const int ft = row_ok ? (K + kTile - 1) / kTile : 0;
     const int nt = ft + (nwin > 0 ? 1 : 0);
     const float scale2 = a.sm_scale * 1.4426950408889634f;  // logits in log2 units
+    uint32_t* status = a.status;
 
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        mbar_init(&bars[kBarS], 1);
+        mbar_init(&bars[kBarO0], 1);
+        mbar_init(&bars[kBarO1], 1);
+        mbar_init(&bars[kBarH0], kT / 2);
+        mbar_init(&bars[kBarH1], kT / 2);
         mbar_fence_init();
     }
     if (tid < 64) s_m[tid] = -INFINITY;
     if (warp == 0) tmem_alloc(tslot, kCols);
+    // the row's indices, checked once (an entry that is -1, not visible or out of range becomes -1)
+    for (int i = tid; i < (row_ok ? K : 0); i += kT) {
+        const int v = __ldg(a.idx + (size_t)row * K + i);
+        const bool ok = v >= 0 && (int64_t)v <= qlast && (int64_t)v < a.c.cap;
+        if (!ok && v != -1) set_status(status, CSA2_DEV_BAD_INDEX);
+        sidx[i] = ok ? v : -1;
+    }
     {   // Q -> fp16 (B operand of S^T, K-major): thread -> head tid >> 3, channels 64 (tid & 7) ..
         const int h = tid >> 3, cb = tid & 7;
         const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)row * kLatHQ + h) * kLatD + 64 * cb);
@@ -163,7 +193,6 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
 
     const size_t seq_row0 = (size_t)b * a.c.cap;
     const size_t swa_row0 = (size_t)b * a.c.swa_cap;
-    uint32_t* status = a.status;
     bool ok_all = true;
     auto wait_bar = [&](int i, uint32_t parity) {
         if (!mbar_wait(&bars[i], parity, kWaitNs)) {
@@ -172,41 +201,42 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
         }
     };
 
+    // this thread's window row (key `key` of the window tile), channels 128 qq ..
+    auto win_src = [&]() {
+        const int64_t p = lo + key;
+        return reinterpret_cast<const uint4*>(a.c.swa + (swa_row0 + (size_t)(p & (a.c.swa_cap - 1))) * kLatSwa +
+                                              128 * qq);
+    };
     // ---- raw rows of tile j into registers (this thread: key `key`, channels 128 qq .. +127) ----
-    uint4 raw[8];
+    // (of a window row only the first 64 channels: the other 64 are loaded while it is dequantised,
+    // so that no more than 18 registers of raw data stay live across the softmax of the tile before)
+    uint4 raw[4];
     uint2 rsc;
     bool kvalid = false;  // the key of this thread in the tile being loaded
     auto load_tile = [&](int j) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) raw[i] = make_uint4(0, 0, 0, 0);
+        for (int i = 0; i < 4; ++i) raw[i] = make_uint4(0, 0, 0, 0);
         rsc = make_uint2(0, 0);
         kvalid = false;
         if (j < ft) {
             const int i = j * kTile + key;
-            if (i < K) {
-                const int v = __ldg(a.idx + (size_t)row * K + i);
-                const bool ok = v >= 0 && (int64_t)v <= qlast && (int64_t)v < a.c.cap;
-                if (!ok && v != -1 && qq == 0) set_status(status, CSA2_DEV_BAD_INDEX);
-                if (ok) {
-                    kvalid = true;
-                    const uint4* src = reinterpret_cast<const uint4*>(a.c.l_data + (seq_row0 + (size_t)v) * kLatBytes + 64 * qq);
+            const int v = i < K ? sidx[i] : -1;
+            if (v >= 0) {
+                kvalid = true;
+                const uint4* src = reinterpret_cast<const uint4*>(a.c.l_data + (seq_row0 + (size_t)v) * kLatBytes + 64 * qq);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
-                    rsc = __ldg(reinterpret_cast<const uint2*>(a.c.l_scale + (seq_row0 + (size_t)v) * kLatScales + 8 * qq));
-                }
+                for (int c = 0; c < 4; ++c) raw[c] = __ldg(src + c);
+                rsc = __ldg(reinterpret_cast<const uint2*>(a.c.l_scale + (seq_row0 + (size_t)v) * kLatScales + 8 * qq));
             }
         } else if (j < nt && key < nwin) {
             kvalid = true;
-            const int64_t p = lo + key;
-            const uint4* src = reinterpret_cast<const uint4*>(
-                a.c.swa + (swa_row0 + (size_t)(p & (a.c.swa_cap - 1))) * kLatSwa + 128 * qq);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) raw[c] = __ldg(src + c);
+            for (int c = 0; c < 4; ++c) raw[c] = __ldg(win_src() + c);  // channels 128 qq .. +63
         }
     };
     // dequantise the registers into the L tile: channel 128 qq + 8 c lands in 64-channel block
     // 2 qq + c / 8, chunk c % 8, of row `key`
-    auto dequant = [&](bool fp4) {
+    auto dequant = [&](bool fp4, bool kvalid_dq) {
         if (fp4) {
 #pragma unroll
             for (int bk = 0; bk < 8; ++bk) {  // 16-channel scale block bk: code words 2 bk, 2 bk + 1
@@ -223,21 +253,31 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
                 *reinterpret_cast<uint4*>(Lt + (2 * qq + ((c0 + 1) >> 3)) * kBlk + sw(key, (c0 + 1) & 7)) = make_uint4(h1[0], h1[1], h1[2], h1[3]);
             }
         } else {
+            // window row: channels 128 qq .. +63 from the registers, then the other 64 channels
+            // (loaded here, once per row, to keep register pressure below the limit)
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {  // 8 window channels per chunk
-                const uint4 rw = raw[c >> 1];
-                const uint32_t w0 = (c & 1) ? rw.z : rw.x, w1 = (c & 1) ? rw.w : rw.y;
-                const uint4 h = make_uint4(e4m3x2_to_h2((uint16_t)(w0 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w0 >> 16)),
-                                           e4m3x2_to_h2((uint16_t)(w1 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w1 >> 16)));
-                *reinterpret_cast<uint4*>(Lt + (2 * qq + (c >> 3)) * kBlk + sw(key, c & 7)) = h;
+            for (int hh = 0; hh < 2; ++hh) {
+                if (hh == 1) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) raw[c] = kvalid_dq ? __ldg(win_src() + 4 + c) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {  // 8 window channels per chunk
+                    const uint4 rw = raw[c >> 1];
+                    const uint32_t w0 = (c & 1) ? rw.z : rw.x, w1 = (c & 1) ? rw.w : rw.y;
+                    const uint4 h = make_uint4(e4m3x2_to_h2((uint16_t)(w0 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w0 >> 16)),
+                                               e4m3x2_to_h2((uint16_t)(w1 & 0xFFFFu)), e4m3x2_to_h2((uint16_t)(w1 >> 16)));
+                    *reinterpret_cast<uint4*>(Lt + (2 * qq + hh) * kBlk + sw(key, c)) = h;
+                }
             }
         }
     };
 
+    __syncthreads();  // barriers, s_m, indices
     load_tile(0);
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();  // barriers, s_m, Q, tensor memory address
+    __syncthreads();  // Q, tensor memory address
     tc_fence_after();
     const uint32_t tb = *tslot;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
@@ -246,41 +286,60 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
 #pragma unroll
     for (int i = 0; i < 16; ++i) lsum[i] = 0.f;
 
+    // Per tile j: each channel half of L is dequantised by its 256 threads as soon as the O^T MMAs
+    // of tile j - 1 that read that half have completed (O^T m-tiles 0, 1 read half 0, m-tiles 2, 3
+    // half 1), and the S^T k-steps of a half are issued as soon as the half is in shared memory, so
+    // that dequantisation overlaps the tensor pipe. The softmax then runs on all 16 warps.
     for (int j = 0; j < nt; ++j) {
         const bool fp4 = j < ft;  // CTA-uniform
         const bool valid = kvalid;
-        if (j > 0) wait_bar(1, (uint32_t)(j - 1) & 1u);  // O^T of tile j - 1 has read L and P
-        dequant(fp4);
-        if (j + 1 < nt) load_tile(j + 1);  // in flight during this tile's MMAs and softmax
+        if (j > 0) wait_bar(half ? kBarO1 : kBarO0, (uint32_t)(j - 1) & 1u);
+        dequant(fp4, valid);
         fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
+        mbar_arrive(&bars[half ? kBarH1 : kBarH0]);
+        if (j + 1 < nt) load_tile(j + 1);  // in flight during this tile's MMAs and softmax
         if (tid == 0) {
+            wait_bar(kBarH0, (uint32_t)j & 1u);
             tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 32; ++kk) {
+            for (int kk = 0; kk < 16; ++kk) {
                 const uint32_t off = (uint32_t)((kk >> 2) * kBlk + 32 * (kk & 3));
                 const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + 32 * (kk & 3));
                 mma_f16(tb + kSCol, sw128_desc(smem_u32(Lt) + off), sw128_desc(smem_u32(Qs) + qoff), kIdescS, kk > 0);
             }
-            mma_commit(&bars[0]);
+            wait_bar(kBarH1, (uint32_t)j & 1u);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 16; kk < 32; ++kk) {
+                const uint32_t off = (uint32_t)((kk >> 2) * kBlk + 32 * (kk & 3));
+                const uint32_t qoff = (uint32_t)((kk >> 2) * kQBlk + 32 * (kk & 3));
+                mma_f16(tb + kSCol, sw128_desc(smem_u32(Lt) + off), sw128_desc(smem_u32(Qs) + qoff), kIdescS, true);
+            }
+            mma_commit(&bars[kBarS]);
         }
-        wait_bar(0, (uint32_t)j & 1u);
+        __syncwarp();
+        wait_bar(kBarS, (uint32_t)j & 1u);  // also every earlier MMA (the O^T of tile j - 1)
         tc_fence_after();
 
         // ---- softmax of the tile: this thread's key 32 quad + lane (= key), heads 16 cg .. +15 ----
-        // (the logits are read from tensor memory twice: for the maxima, then for P, which keeps
-        // them out of registers during the reduction)
-        const uint32_t s_addr = tb + lane_base + kSCol + 16 * cg;
+        float lg[16];  // raw logits q . l (the scale is applied inside the exponent)
         {
             uint32_t v[16];
-            tmem_ld16(s_addr, v);
+            tmem_ld16(tb + lane_base + kSCol + 16 * cg, v);
             tmem_ld_wait();
-            float mx[16];
+            float r[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) mx[i] = valid ? __uint_as_float(v[i]) * scale2 : -INFINITY;
-            const float r = warp_reduce16<true>(mx, lane);
-            if (lane < 16) red[quad * 64 + 16 * cg + lane] = r;
+            for (int i = 0; i < 16; ++i) {
+                lg[i] = __uint_as_float(v[i]);
+                r[i] = warp_max(valid ? lg[i] * scale2 : -INFINITY);  // (any sign of the scale)
+            }
+            if (lane == 0) {
+                float4* d = reinterpret_cast<float4*>(red + quad * 64 + 16 * cg);
+                d[0] = make_float4(r[0], r[1], r[2], r[3]);
+                d[1] = make_float4(r[4], r[5], r[6], r[7]);
+                d[2] = make_float4(r[8], r[9], r[10], r[11]);
+                d[3] = make_float4(r[12], r[13], r[14], r[15]);
+            }
         }
         __syncthreads();
         int resc = 0;
@@ -299,7 +358,7 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
         const float* al = s_al + 16 * cg;  // this warp's heads (shared-memory broadcasts)
         const float* mh = s_m + 16 * cg;
         if (resc) {
-            // O^T (columns = heads) of tile j - 1 is complete: scale this warp's heads in place
+            // every O^T MMA so far has completed (the S^T commit tracks them): scale in place
 #pragma unroll
             for (int mt = 0; mt < 4; ++mt) {
                 uint32_t v[16];
@@ -312,22 +371,14 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
             }
             tmem_st_wait();
         }
+        // a valid key makes every head's maximum finite, so p needs no test of m for -inf
         uint32_t ph[8];
-        float lg[16];
-        {
-            uint32_t v[16];
-            tmem_ld16(s_addr, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) lg[i] = valid ? __uint_as_float(v[i]) * scale2 : -INFINITY;
-        }
 #pragma unroll
         for (int i = 0; i < 16; i += 2) {
-            const float m0 = mh[i], m1 = mh[i + 1];
-            const float p0 = (m0 == -INFINITY) ? 0.f : exp2f(lg[i] - m0);
-            const float p1 = (m1 == -INFINITY) ? 0.f : exp2f(lg[i + 1] - m1);
-            lsum[i] = lsum[i] * al[i] + p0;
-            lsum[i + 1] = lsum[i + 1] * al[i + 1] + p1;
+            const float p0 = valid ? ex2(fmaf(lg[i], scale2, -mh[i])) : 0.f;
+            const float p1 = valid ? ex2(fmaf(lg[i + 1], scale2, -mh[i + 1])) : 0.f;
+            lsum[i] = fmaf(lsum[i], al[i], p0);
+            lsum[i + 1] = fmaf(lsum[i + 1], al[i + 1], p1);
             ph[i >> 1] = pack_h2(p0, p1);
         }
         // P [key][head]: heads 16 cg .. +7 -> chunk 2 cg, 16 cg + 8 .. -> chunk 2 cg + 1
@@ -348,31 +399,25 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
                     const uint64_t bd = sw128_desc_mn(smem_u32(Ps) + (uint32_t)(2048 * kk), 0);
                     mma_f16(tb + kOCol + 64 * mt, ad, bd, kIdescO, j > 0 || kk > 0);
                 }
+                if (mt == 1) mma_commit(&bars[kBarO0]);  // channel half 0 of L is free again
             }
-            mma_commit(&bars[1]);
+            mma_commit(&bars[kBarO1]);
         }
+        __syncwarp();
     }
     if (nt > 0) {
-        wait_bar(1, (uint32_t)(nt - 1) & 1u);
+        wait_bar(kBarO1, (uint32_t)(nt - 1) & 1u);  // the last MMAs (in issue order)
         tc_fence_after();
     }
 
     // ---- epilogue: l per head, then out = O / l (warp: channels 128 mt + 32 quad + lane, heads 16 cg ..) ----
     {
-        const float r = warp_reduce16<false>(lsum, lane);
+        const float r = warp_sum16(lsum, lane);
         if (lane < 16) red[quad * 64 + 16 * cg + lane] = r;
     }
     __syncthreads();
     if (tid < 64) s_l[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
     __syncthreads();
-    float inv[16];
-    bool empty[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int h = 16 * cg + i;
-        empty[i] = (nt == 0) || (s_m[h] == -INFINITY) || !(s_l[h] > 0.f);
-        inv[i] = empty[i] ? 0.f : 1.f / s_l[h];
-    }
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
         uint32_t v[16] = {};
@@ -383,7 +428,9 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
         const int d = 128 * mt + 32 * quad + lane;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const float x = empty[i] ? 0.f : __uint_as_float(v[i]) * inv[i];
+            const int h = 16 * cg + i;
+            const bool em = (nt == 0) || (s_m[h] == -INFINITY) || !(s_l[h] > 0.f);
+            const float x = em ? 0.f : __uint_as_float(v[i]) * (1.f / s_l[h]);
             const size_t ob = ((size_t)row * kLatHQ + 16 * cg + i) * kLatD + d;
             a.out[ob] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
             if (a.out_f32) a.out_f32[ob] = x;
