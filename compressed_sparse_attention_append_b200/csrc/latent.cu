@@ -170,25 +170,20 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
     }
     if (tid < 64) s_m[tid] = -INFINITY;
     if (warp == 0) tmem_alloc(tslot, kCols);
+    // Q (this thread: head tid >> 3, channels 64 (tid & 7) ..) requested first; it is converted once
+    // the row's indices are staged and tile 0's rows requested, so that the three loads overlap
+    uint4 qv[8];
+    {
+        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)row * kLatHQ + (tid >> 3)) * kLatD + 64 * (tid & 7));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) qv[c] = __ldg(src + c);
+    }
     // the row's indices, checked once (an entry that is -1, not visible or out of range becomes -1)
     for (int i = tid; i < (row_ok ? K : 0); i += kT) {
         const int v = __ldg(a.idx + (size_t)row * K + i);
         const bool ok = v >= 0 && (int64_t)v <= qlast && (int64_t)v < a.c.cap;
         if (!ok && v != -1) set_status(status, CSA2_DEV_BAD_INDEX);
         sidx[i] = ok ? v : -1;
-    }
-    {   // Q -> fp16 (B operand of S^T, K-major): thread -> head tid >> 3, channels 64 (tid & 7) ..
-        const int h = tid >> 3, cb = tid & 7;
-        const uint4* src = reinterpret_cast<const uint4*>(a.q + ((size_t)row * kLatHQ + h) * kLatD + 64 * cb);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const uint4 x = __ldg(src + c);
-            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-            uint32_t hv[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) hv[i] = pack_h2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-            *reinterpret_cast<uint4*>(Qs + cb * kQBlk + sw(h, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-        }
     }
 
     const size_t seq_row0 = (size_t)b * a.c.cap;
@@ -275,6 +270,17 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
 
     __syncthreads();  // barriers, s_m, indices
     load_tile(0);
+    {   // Q -> fp16 (B operand of S^T, K-major: row = head, 64-channel blocks)
+        const int h = tid >> 3, cb = tid & 7;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const uint32_t w[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
+            uint32_t hv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hv[i] = pack_h2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+            *reinterpret_cast<uint4*>(Qs + cb * kQBlk + sw(h, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+        }
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();  // Q, tensor memory address
@@ -416,7 +422,12 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
         if (lane < 16) red[quad * 64 + 16 * cg + lane] = r;
     }
     __syncthreads();
-    if (tid < 64) s_l[tid] = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
+    if (tid < 64) {
+        const float l = (red[tid] + red[64 + tid]) + (red[128 + tid] + red[192 + tid]);
+        s_l[tid] = l;
+        const bool em = (nt == 0) || (s_m[tid] == -INFINITY) || !(l > 0.f);
+        s_al[tid] = em ? 0.f : 1.f / l;  // 1 / l per head (0 for a row with no key: O is 0 there)
+    }
     __syncthreads();
 #pragma unroll
     for (int mt = 0; mt < 4; ++mt) {
@@ -428,9 +439,7 @@ __global__ void __launch_bounds__(kT, 1) latent_attend_kernel(LatentAttendArgs a
         const int d = 128 * mt + 32 * quad + lane;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            const int h = 16 * cg + i;
-            const bool em = (nt == 0) || (s_m[h] == -INFINITY) || !(s_l[h] > 0.f);
-            const float x = em ? 0.f : __uint_as_float(v[i]) * (1.f / s_l[h]);
+            const float x = __uint_as_float(v[i]) * s_al[16 * cg + i];
             const size_t ob = ((size_t)row * kLatHQ + 16 * cg + i) * kLatD + d;
             a.out[ob] = __bfloat16_as_ushort(__float2bfloat16_rn(x));
             if (a.out_f32) a.out_f32[ob] = x;
