@@ -40,6 +40,10 @@ def algorithmic_bytes(wl):
         # the pages' own shape: k selected latent entries (256 B codes + 32 B scales), the window rows
         # (512 B), the query and the output (64 heads x 512, bf16) and the indices, per row
         return {"append": 0, "index": 0, "attend": k * 288 + win * 512 + 2 * (64 * 512 * 2) + k * 4}
+    if wl.mode == "latent_index":
+        # the pages' own indexer: every visible MXFP4 key (64 B codes + 4 B scales), the query
+        # (hi x 128 bf16), its position and the selected indices, per row
+        return {"append": 0, "index": wl.context * 68 + wl.hi * 128 * 2 + 8 + k * 4, "attend": 0}
     q, out, iq, idx = 16 * 128 * 2, 16 * 128 * 2, 4 * 64 * 2, k * 4
     attend = k * 144 + win * 256 + q + idx + out
     if wl.mode == "reindex":
@@ -84,6 +88,8 @@ def kernels_per_step(wl):
     attention 1."""
     if wl.mode == "latent":
         return 1
+    if wl.mode == "latent_index":
+        return 3
     if wl.mode == "minimal":
         return 2
     if wl.mode in ("full", "reindex"):
@@ -515,6 +521,9 @@ def run_gpu(args):
     if wl.mode == "latent":
         kms.pop("index", None)
         kms.pop("append", None)
+    if wl.mode == "latent_index":
+        kms.pop("attend", None)
+        kms.pop("append", None)
 
     # ---- end to end: host inputs -> C ABI call -> host outputs ----
     e2e = run_e2e(step, args, world, barrier)
@@ -566,7 +575,9 @@ def run_gpu(args):
     else:
         dom_bytes = ab[dom] * B
         # decode rows: the index step is zero_kernel + score_kernel + select_kernel (index_decode.cu)
-        if dom == "index":
+        if wl.mode == "latent_index":
+            dom_file, dom_kernels = "latent_index.cu", "mxfp4_kernel + lat_index_score_kernel + lat_index_select_kernel"
+        elif dom == "index":
             dom_file, dom_kernels = "index_decode.cu", "zero_kernel + score_kernel + select_kernel"
         elif wl.mode == "latent":
             dom_file, dom_kernels = "latent.cu", "latent_attend_kernel"
@@ -598,9 +609,12 @@ def run_gpu(args):
                    "batch_per_gpu": B, "query_rows_per_sequence": wl.tq, "context": wl.context,
                    "pool_blocks": wl.pool_blocks, "topk": wl.k, "query_heads": wl.hq, "head_dim": wl.d,
                    "indexer": ("none in the step (inherited selection)" if wl.mode == "latent" else
-                               "4 heads x 64, FP4"),
+                               f"{wl.hi} heads x 128 over one MXFP4 key per entry, ReLU scores"
+                               if wl.mode == "latent_index" else "4 heads x 64, FP4"),
                    "kv_cache": ("one 512-channel latent per entry (K = V), E2M1 + E4M3/16, window FP8 x 512"
-                                if wl.mode == "latent" else "E2M1 + E4M3/16 (FP4), window FP8"),
+                                if wl.mode == "latent" else
+                                "MXFP4 indexer key only (E2M1 + E8M0/32, 68 B per entry)"
+                                if wl.mode == "latent_index" else "E2M1 + E4M3/16 (FP4), window FP8"),
                    "window": wl.win, "parallelism": f"dp{world}",
                    "l2": (f"L2 flushed between timed steps (a step reads {step_bytes / 1e6:.0f} MB, less than the L2)"
                           if flush else f"inputs larger than L2 ({step_bytes / 1e6:.0f} MB read per step)"),
@@ -656,7 +670,7 @@ def run_e2e(step, args, world, barrier):
     else:
         names_in = [n for n in ("pos", "qpos", "swa_kv", "idx_q", "q", "pool", "pool_n", "kv", "idx_k", "idx")
                     if n in step.inputs]
-    names_out = ["out"] + (["idx"] if "idx" in step.outputs and wl.mode != "minimal" else [])
+    names_out = [n for n in ("out", "idx") if n in step.outputs and not (n == "idx" and wl.mode == "minimal")]
     dev = step.inputs[names_in[0]].device
     slots = []
     for _ in range(2):
@@ -728,6 +742,8 @@ def e2e_call(mode):
     """The public entry point(s) one end-to-end step goes through."""
     if mode == "latent":
         return "csa2_latent_attend"
+    if mode == "latent_index":
+        return "csa2_latent_index_topk"
     if mode == "prefill":
         return "csa2_prefill_chunk"
     if mode == "draft":

@@ -49,7 +49,7 @@ EXPORTS = (
     "csa2_quantize_append", "csa2_index_topk_full", "csa2_index_topk_reindex", "csa2_sparse_attend",
     "csa2_decode_full", "csa2_decode_reindex", "csa2_decode_minimal", "csa2_prefill_chunk",
     "csa2_get_device_status", "csa2_sparse_attend_noalloc", "csa2_mx_entry_bytes", "csa2_mxfp4_quantize",
-    "csa2_latent_append", "csa2_latent_attend",
+    "csa2_latent_append", "csa2_latent_attend", "csa2_latent_index_workspace_size", "csa2_latent_index_topk",
 )
 
 
@@ -112,6 +112,8 @@ def lib():
             "csa2_mxfp4_quantize": (i, [vp, i64, i, vp, vp, vp]),
             "csa2_latent_append": (i, [LC, i, i, vp, vp, vp, vp, vp, sz, vp]),
             "csa2_latent_attend": (i, [LC, i, i, vp, vp, vp, i, vp, i, i, f, vp, vp, vp, vp, sz, vp]),
+            "csa2_latent_index_workspace_size": (i, [i, i, i64, ctypes.POINTER(sz)]),
+            "csa2_latent_index_topk": (i, [LC, i, i, vp, vp, i, i, i, i64, u32, vp, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -208,12 +210,12 @@ class LatentCache:
     sequences: the 512-channel latent (E2M1 + E4M3 per 16), the 128-channel MXFP4 indexer key and
     a ring of 512-channel E4M3 window rows, allocated with torch."""
 
-    def __init__(self, batch: int, cap: int, swa_cap: int = 128, device="cuda", indexer=True):
+    def __init__(self, batch: int, cap: int, swa_cap: int = 128, device="cuda", indexer=True, latent=True):
         assert swa_cap & (swa_cap - 1) == 0
         self.batch, self.cap, self.swa_cap = batch, cap, swa_cap
         z = lambda *s: torch.zeros(*s, dtype=torch.uint8, device=device)
-        self.l_data = z(batch, cap, 256)
-        self.l_scale = z(batch, cap, 32)
+        self.l_data = z(batch, cap, 256) if latent else None
+        self.l_scale = z(batch, cap, 32) if latent else None
         self.k_data = z(batch, cap, 64) if indexer else None
         self.k_scale = z(batch, cap, 4) if indexer else None
         self.swa = z(batch, swa_cap, 512)
@@ -238,6 +240,40 @@ def csa2_latent_attend(cache: LatentCache, batch, tq, qpos, q, idx, k, out, swa_
     _check("csa2_latent_attend", lib().csa2_latent_attend(
         cache.ref, batch, tq, _i64(qpos), _bits(q), _i32(idx), k, _i64(swa_begin), win, ratio, sm_scale, _bits(out),
         _f32(out_f32), _f32(lse), ws.ptr if ws else None, ws.nbytes if ws else 0, _stream(stream)))
+
+
+def csa2_latent_index_workspace_size(rows, hi, max_ctx) -> int:
+    out = ctypes.c_size_t(0)
+    _check("csa2_latent_index_workspace_size",
+           lib().csa2_latent_index_workspace_size(rows, hi, max_ctx, ctypes.byref(out)))
+    return out.value
+
+
+class LatentIndexWorkspace:
+    """Workspace of csa2_latent_index_topk for `rows` query rows of `hi` heads and at most `max_ctx`
+    visible entries per row (zeroed: its first word is the status word)."""
+
+    def __init__(self, rows, hi, max_ctx, device="cuda"):
+        self.buf = torch.zeros(csa2_latent_index_workspace_size(rows, hi, max_ctx), dtype=torch.uint8, device=device)
+        assert self.buf.data_ptr() % 256 == 0
+
+    @property
+    def ptr(self):
+        return self.buf.data_ptr()
+
+    @property
+    def nbytes(self):
+        return self.buf.numel()
+
+
+def csa2_latent_index_topk(cache: LatentCache, batch, tq, qpos, idx_q, k, out_idx, ws, ratio=1, max_ctx=None,
+                           flags=0, stream=None):
+    """idx_q [B*tq, hi, 128] bf16 -> out_idx [B*tq, k] int32 (the indexer of the pages' own shape)."""
+    if max_ctx is None:
+        max_ctx = cache.cap
+    _check("csa2_latent_index_topk", lib().csa2_latent_index_topk(
+        cache.ref, batch, tq, _i64(qpos), _bits(idx_q), idx_q.shape[-2], k, ratio, max_ctx, flags, _i32(out_idx),
+        ws.ptr, ws.nbytes, _stream(stream)))
 
 
 def csa2_entry_bytes(channels: int) -> int:

@@ -7,7 +7,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = [os.path.join(HERE, "csrc", f) for f in ("abi.cu", "append.cu", "index.cu", "index_decode.cu", "index_mma.cu", "attend.cu", "noalloc.cu", "latent.cu")]
+SRC = [os.path.join(HERE, "csrc", f) for f in ("abi.cu", "append.cu", "index.cu", "index_decode.cu", "index_mma.cu", "attend.cu", "noalloc.cu", "latent.cu", "latent_index.cu")]
 HDRS = [os.path.join(HERE, "csrc", "csa2_internal.cuh"), os.path.join(HERE, "csrc", "tc.cuh"), os.path.join(ROOT, "include", "csa2.h")]
 LIB = os.path.join(HERE, "libcsa2.so")
 

@@ -1,7 +1,7 @@
 // abi.cu -- the extern "C" entry points of libcsa2 (declared and documented in include/csa2.h):
 // argument validation, workspace planning, kernel launches, status codes. Nothing here computes
 // any part of the layer step; every step runs in the kernels of append.cu, index.cu, index_decode.cu,
-// index_mma.cu, attend.cu, noalloc.cu and latent.cu.
+// index_mma.cu, attend.cu, noalloc.cu, latent.cu and latent_index.cu.
 #include <math.h>
 
 #include "csa2_internal.cuh"
@@ -240,6 +240,39 @@ csa2_status csa2_latent_attend(const csa2_latent_cache* cache, int batch, int tq
     a.lse = lse;
     a.status = ws ? reinterpret_cast<uint32_t*>(ws) : nullptr;
     return from_cuda(launch_latent_attend(a, (cudaStream_t)stream));
+}
+
+csa2_status csa2_latent_index_workspace_size(int rows, int hi, int64_t max_ctx, size_t* bytes) {
+    if (!bytes || rows < 0 || rows > 65535 || hi < 1 || hi > kLatMaxHI || max_ctx < 1) return CSA2_ERR_INVALID_ARG;
+    *bytes = latent_index_ws_bytes(rows, hi, max_ctx);
+    return CSA2_OK;
+}
+
+csa2_status csa2_latent_index_topk(const csa2_latent_cache* cache, int batch, int tq, const int64_t* qpos,
+                                   const uint16_t* idx_q, int hi, int k, int ratio, int64_t max_ctx, uint32_t flags,
+                                   int32_t* out_idx, void* ws, size_t ws_bytes, void* stream) {
+    if (!cache || !qpos || !idx_q || !out_idx || !ws || batch < 0 || tq < 1) return CSA2_ERR_INVALID_ARG;
+    if (hi < 1 || hi > kLatMaxHI || k < 1 || k > kMaxK || max_ctx < 1) return CSA2_ERR_INVALID_ARG;
+    if (ratio != 1 && ratio != 2) return CSA2_ERR_UNSUPPORTED_SHAPE;
+    if ((long long)batch * tq > 65535) return CSA2_ERR_INVALID_ARG;
+    if (cache->cap <= 0 || cache->cap > ((int64_t)1 << 30)) return CSA2_ERR_INVALID_ARG;
+    if (!cache->k_data || !cache->k_scale || !al16(cache->k_data) || !al16(cache->k_scale)) return CSA2_ERR_INVALID_ARG;
+    if (!al16(idx_q) || ((uintptr_t)ws & 255u)) return CSA2_ERR_INVALID_ARG;
+    const int rows = batch * tq;
+    if (ws_bytes < latent_index_ws_bytes(rows, hi, max_ctx)) return CSA2_ERR_WORKSPACE;
+    if (rows == 0) return CSA2_OK;
+    LatIndexArgs a{};
+    a.c = *cache;
+    a.rows = rows;
+    a.tq = tq;
+    a.hi = hi;
+    a.k = k;
+    a.ratio = ratio;
+    a.max_ctx = max_ctx;
+    a.qpos = qpos;
+    a.flags = flags;
+    a.out_idx = out_idx;
+    return from_cuda(launch_latent_index(a, idx_q, reinterpret_cast<unsigned char*>(ws), (cudaStream_t)stream));
 }
 
 const char* csa2_status_string(csa2_status s) {

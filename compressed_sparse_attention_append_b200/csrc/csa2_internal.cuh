@@ -518,4 +518,21 @@ struct LatentAttendArgs {
 size_t latent_attend_smem_bytes();
 cudaError_t launch_latent_attend(const LatentAttendArgs& a, cudaStream_t s);
 
+constexpr int kLatMaxHI = 64;    // indexer query heads the latent indexer takes
+struct LatIndexArgs {
+    csa2_latent_cache c;
+    int rows, tq, hi, k, ratio;
+    int64_t max_ctx;              // bound on a row's visible entries (the key buffer's row length)
+    const int64_t* qpos;          // [rows]
+    uint32_t flags;
+    const uint8_t* qcodes;        // workspace: the rows' quantised queries [rows][hi][64]
+    const uint8_t* qscales;       // [rows][hi][4]
+    unsigned long long* keys;     // [rows][max_ctx] orderable score keys
+    int64_t key_stride;
+    int32_t* out_idx;
+    uint32_t* status;
+};
+size_t latent_index_ws_bytes(int rows, int hi, int64_t max_ctx);
+cudaError_t launch_latent_index(LatIndexArgs a, const uint16_t* idx_q, unsigned char* ws, cudaStream_t s);
+
 }  // namespace csa2

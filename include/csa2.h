@@ -353,6 +353,29 @@ CSA2_API csa2_status csa2_latent_attend(const csa2_latent_cache* cache, int batc
                                         int win, int ratio, float sm_scale, uint16_t* out, float* out_f32, float* lse,
                                         void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Indexer of the pages' own shape ([C] sec. VII: the indexer key is ONE 128-channel MXFP4 key per
+ * entry; the configuration list: 32 indexer query heads of dimension 128; [B] "Technical Approach",
+ * [C] sec. VI: Top-k of the visible entries). For each of the batch*tq query rows:
+ *   idx_q [batch*tq][hi][128] bf16 (16-byte aligned), 1 <= hi <= 64, quantised on the device with
+ *   the MXFP4 rule of csa2_mxfp4_quantize; keys from cache->k_data / k_scale of sequence row / tq;
+ *   score(p) = sum_h q_h . k_p, or sum_h max(0, q_h . k_p) with flags & CSA2_SCORE_RELU (the
+ *   reading taken here; the pages give no formula) over the (qpos + 1) / ratio visible entries;
+ *   out_idx [batch*tq][k]: the Top-k by score descending, ties to the lower position, in ascending
+ *   position order, padded with -1 (a row with qpos < 0 gives all -1).
+ * Scores are evaluated exactly (integer block dots times power-of-two scales, fp64 sums) whenever
+ * the 32-channel block maxima of a row's query and keys lie within 2^38 of each other.
+ * ws: at least csa2_latent_index_workspace_size(batch*tq, hi, max_ctx) bytes, 256-byte aligned
+ * (its first 4 bytes are the status word; the rest is scratch); max_ctx bounds the visible
+ * entries of every row: a row with more, or whose entries run past the capacity, sets
+ * CSA2_DEV_BAD_POS and gives all -1. batch*tq <= 65535, 1 <= k <= 2048, ratio 1 or 2.
+ */
+CSA2_API csa2_status csa2_latent_index_workspace_size(int rows, int hi, int64_t max_ctx, size_t* bytes /* host */);
+CSA2_API csa2_status csa2_latent_index_topk(const csa2_latent_cache* cache, int batch, int tq, const int64_t* qpos,
+                                            const uint16_t* idx_q, int hi, int k, int ratio, int64_t max_ctx,
+                                            uint32_t flags, int32_t* out_idx, void* ws, size_t ws_bytes,
+                                            void* stream);
+
 /* Synchronises `stream`, then reads and clears the device status word in `ws`.
  * *host_status receives the CSA2_DEV_* bits; returns CSA2_ERR_DEVICE if any bit was set. */
 CSA2_API csa2_status csa2_get_device_status(void* ws, void* stream, int32_t* host_status /* host */);

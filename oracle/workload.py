@@ -26,6 +26,13 @@ def build_sequence(wl, b):
     """Returns (cache, inputs) of sequence b before its step."""
     N, seed = wl.context, wl.seed
     inp = {}
+    if wl.mode == "latent_index":
+        # the pages' own indexer: the MXFP4 key of every visible entry
+        c = LatentCache(cap=N, swa_cap=128)
+        for a in range(0, N, 16384):
+            c.append(a, idx_k=_v(seed, "lik", b, torch.arange(a, min(N, a + 16384)), 128))
+        inp["idx_q"] = _v(seed, "liq", b, [N - 1], wl.hi * 128)[0].reshape(wl.hi, 128)
+        return c, inp
     if wl.mode == "latent":
         # the pages' own shape: the latent rows of the selected entries and the window rows
         c = LatentCache(cap=N, swa_cap=128)
@@ -101,6 +108,9 @@ def run_step(c, wl, inp, rows=None):
     rows = {row: (idx, out, lse)}."""
     N = wl.context
     r = {}
+    if wl.mode == "latent_index":
+        r["idx"], _ = c.index_topk_full(N - 1, inp["idx_q"], k=wl.k, relu=True)
+        return r
     if wl.mode == "latent":
         r["idx"] = inp["idx"]
         r["out"], r["lse"] = c.attend(N - 1, inp["q"], inp["idx"], win=wl.win)

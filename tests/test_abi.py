@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(L):
     names = declared_symbols()
-    assert len(names) == 19
+    assert len(names) == 21
     assert set(names) == set(csa.EXPORTS)
     for n in names:
         assert hasattr(L, n), n
@@ -278,3 +278,33 @@ def test_latent_entry_points_validate_before_any_launch(L):
     assert app(rc, 1, 2048, qpos, x, None, None, None, 0, None) == csa.CSA2_ERR_CAPACITY
     nokey = csa.csa2_latent_cache(base, base + 4096, None, None, base + 16384, 1024, 128)
     assert app(ctypes.byref(nokey), 1, 1, qpos, None, x, None, None, 0, None) == csa.CSA2_ERR_INVALID_ARG
+
+
+def test_latent_index_entry_points_validate_before_any_launch(L):
+    """The indexer of the pages' own shape: workspace sizing and argument checks on the host; an
+    empty batch returns OK without a launch."""
+    sz = ctypes.c_size_t(0)
+    assert L.csa2_latent_index_workspace_size(4, 32, 1000, ctypes.byref(sz)) == csa.CSA2_OK
+    # status line, 4 x 32 query codes (64 B) and scales (4 B), 4 x 1000 8-byte keys, 256-byte aligned parts
+    assert sz.value == 256 + 8192 + 512 + 32000
+    for bad in ((4, 0, 1000), (4, 65, 1000), (-1, 32, 1000), (70000, 32, 1000), (4, 32, 0)):
+        assert L.csa2_latent_index_workspace_size(*bad, ctypes.byref(sz)) == csa.CSA2_ERR_INVALID_ARG
+    buf = ctypes.create_string_buffer(1 << 16)
+    base = (ctypes.addressof(buf) + 255) & ~255
+    c = csa.csa2_latent_cache(None, None, base + 8192, base + 12288, None, 1024, 128)
+    rc = ctypes.byref(c)
+    f = L.csa2_latent_index_topk
+    qpos = iq = out = base + 16384
+    ws = base + 32768
+    # (cache, batch, tq, qpos, idx_q, hi, k, ratio, max_ctx, flags, out_idx, ws, ws_bytes, stream)
+    assert f(rc, 0, 1, qpos, iq, 32, 512, 1, 1000, 0, out, ws, 256, None) == csa.CSA2_OK
+    assert f(rc, 1, 1, qpos, iq, 32, 512, 1, 1000, 0, out, ws, 256, None) == csa.CSA2_ERR_WORKSPACE
+    assert f(rc, 1, 1, qpos, iq, 0, 512, 1, 1000, 0, out, ws, 1 << 20, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(rc, 1, 1, qpos, iq, 32, 4096, 1, 1000, 0, out, ws, 1 << 20, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(rc, 1, 1, qpos, iq, 32, 512, 3, 1000, 0, out, ws, 1 << 20, None) == csa.CSA2_ERR_UNSUPPORTED_SHAPE
+    assert f(rc, 1, 1, qpos, iq + 2, 32, 512, 1, 1000, 0, out, ws, 1 << 20, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(rc, 1, 1, qpos, iq, 32, 512, 1, 1000, 0, out, ws + 16, 1 << 20, None) == csa.CSA2_ERR_INVALID_ARG
+    assert f(None, 1, 1, qpos, iq, 32, 512, 1, 1000, 0, out, ws, 1 << 20, None) == csa.CSA2_ERR_INVALID_ARG
+    nokey = csa.csa2_latent_cache(None, None, None, None, None, 1024, 128)
+    assert f(ctypes.byref(nokey), 1, 1, qpos, iq, 32, 512, 1, 1000, 0, out, ws, 1 << 20, None) == \
+        csa.CSA2_ERR_INVALID_ARG

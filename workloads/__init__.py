@@ -42,8 +42,9 @@ _C1 = _s64(0xBF58476D1CE4E5B9)
 _C2 = _s64(0x94D049BB133111EB)
 
 STREAM = {"kv": 1, "ik": 2, "swa": 3, "q": 4, "iq": 5, "pool": 6, "sel": 7,
-          # the pages' own shape: 512-channel latent, 128-channel indexer key, window rows, query
-          "lat": 8, "lik": 9, "lsw": 10, "lq": 11}
+          # the pages' own shape: 512-channel latent, 128-channel indexer key, window rows, query,
+          # indexer query
+          "lat": 8, "lik": 9, "lsw": 10, "lq": 11, "liq": 12}
 POS_BITS = 21  # positions per sequence addressed by the counters: < 2^21
 
 
@@ -115,7 +116,7 @@ def distinct_sorted(seed: int, stream, b: torch.Tensor, n_range: int, count: int
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    mode: str            # "full" | "reindex" | "minimal" | "prefill" | "draft" | "latent"
+    mode: str            # "full" | "reindex" | "minimal" | "prefill" | "draft" | "latent" | "latent_index"
     batch: int
     context: int         # N: visible positions for a decode query (query at N-1)
     seed: int
@@ -144,4 +145,8 @@ WORKLOADS = {
     # the pages' own attention shape: 64 query heads x 512 over the 512-channel latent (K = V), a
     # decode row per sequence at N - 1 with 512 inherited selected entries and a 128-token window
     "latent_b128_n131072": Workload("latent_b128_n131072", "latent", 128, 131072, seed=6, hq=64, d=512),
+    # the pages' own indexer: 32 query heads x 128 over one 128-channel MXFP4 key per entry, ReLU
+    # scores, Top-512 of every visible entry, a decode row per sequence at N - 1
+    "latent_index_b128_n131072": Workload("latent_index_b128_n131072", "latent_index", 128, 131072, seed=7, hi=32,
+                                          di=128),
 }

@@ -183,6 +183,45 @@ def _build_latent(wl, seqs, B, device):
     return LatentStep(wl, cache, ws, {"qpos": qpos, "q": q, "idx": idx}, {"out": out}, B)
 
 
+@dataclasses.dataclass
+class LatentIndexStep:
+    """A decode row per sequence scored by the indexer of the pages' own shape (32 heads x 128 over
+    one MXFP4 key per entry, ReLU scores) against every visible entry: one csa2_latent_index_topk."""
+    wl: Workload
+    cache: csa.LatentCache
+    ws: csa.LatentIndexWorkspace
+    inputs: dict
+    outputs: dict
+    batch: int
+
+    def run(self, stream=None, ws=None, out_f32=None, lse=None):
+        I, O = self.inputs, self.outputs
+        csa.csa2_latent_index_topk(self.cache, self.batch, 1, I["qpos"], I["idx_q"], self.wl.k, O["idx"], ws or self.ws,
+                                   max_ctx=self.wl.context, flags=csa.CSA2_SCORE_RELU, stream=stream)
+
+    def run_parts(self, hooks, stream=None):
+        hooks("index", 0)
+        self.run(stream)
+        hooks("index", 1)
+
+
+def _build_latent_index(wl, seqs, B, device, chunk=4096):
+    N = wl.context
+    cache = csa.LatentCache(B, N, 128, device=device, latent=False)
+    st = StatusWs(device)
+    for p0 in range(0, N, chunk):  # every position: the step scans them all
+        t = min(chunk, N - p0)
+        p = torch.arange(p0, p0 + t, device=device)
+        csa.csa2_latent_append(cache, B, t, torch.full((B,), p0, dtype=torch.int64, device=device),
+                               idx_k=_vals(wl.seed, "lik", seqs, p, 128).contiguous(), ws=st)
+    qpos = torch.full((B,), N - 1, dtype=torch.int64, device=device)
+    iq = _vals(wl.seed, "liq", seqs, qpos.unsqueeze(1), wl.hi * 128)[:, 0].reshape(B, wl.hi, 128).contiguous()
+    out = torch.empty(B, wl.k, dtype=torch.int32, device=device)
+    ws = csa.LatentIndexWorkspace(B, wl.hi, N, device=device)
+    torch.cuda.synchronize()
+    return LatentIndexStep(wl, cache, ws, {"qpos": qpos, "idx_q": iq}, {"idx": out}, B)
+
+
 def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda", context=None) -> Step:
     """Allocate and fill the cache of workload `name` (optionally a smaller batch, or the sequences
     seq_offset .. seq_offset+batch-1 of it, as a data-parallel rank would; optionally another context
@@ -194,6 +233,8 @@ def build(name: str, batch: int | None = None, seq_offset: int = 0, device="cuda
     seqs = torch.arange(seq_offset, seq_offset + B, device=device)
     if wl.mode == "latent":
         return _build_latent(wl, seqs, B, device)
+    if wl.mode == "latent_index":
+        return _build_latent_index(wl, seqs, B, device)
     shape = csa.make_shape(wl.win)
     N = wl.context
     I, O = {}, {}
