@@ -158,3 +158,20 @@ def test_draft_rows_share_one_pass_over_the_keys():
     assert ab["index"] * wl.tq == 131072 * 144 + 5 * (4 * 64 * 2 + 512 * 4)
     assert bench.e2e_call("draft").startswith("csa2_quantize_append")
     assert bench.e2e_call("reindex") == "csa2_decode_reindex"
+
+
+def test_latent_workloads_bytes_flops_and_calls():
+    """The pages' own shapes: the latent attention reads k latent entries (256 + 32 B), the window
+    rows (512 B), q and writes out (64 x 512 bf16 each) and reads the indices; its two contractions
+    take 2 x 2 x 64 x 512 flops per key. The indexer reads every visible MXFP4 key (68 B), its query
+    (32 x 128 bf16) and position, and writes k indices."""
+    import workloads as W
+
+    wl = W.WORKLOADS["latent_b128_n131072"]
+    assert bench.algorithmic_bytes(wl) == {"append": 0, "index": 0, "attend": 346112}
+    assert 512 * 288 + 128 * 512 + 2 * 65536 + 2048 == 346112
+    assert bench.latent_flops(wl) == 4 * 64 * 512 * 640
+    assert bench.kernels_per_step(wl) == 1 and bench.e2e_call("latent") == "csa2_latent_attend"
+    wi = W.WORKLOADS["latent_index_b128_n131072"]
+    assert bench.algorithmic_bytes(wi)["index"] == 131072 * 68 + 32 * 128 * 2 + 8 + 512 * 4
+    assert bench.kernels_per_step(wi) == 3 and bench.e2e_call("latent_index") == "csa2_latent_index_topk"
