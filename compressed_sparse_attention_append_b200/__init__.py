@@ -20,6 +20,15 @@ A Reindex decode step for a batch of B sequences (tensors on the GPU, bf16 unles
 `out` [B, 16, 128] holds the attention output, `idx` [B, 512] the selected positions (ascending,
 -1 padded). The Full and Minimal modes, the separate index / attention calls and the prefill chunk
 follow the same pattern (include/csa2.h documents every argument).
+
+The pages' own shapes use a `LatentCache` (one 512-channel latent per entry that is both key and
+value, a 128-channel MXFP4 indexer key, 512-channel FP8 window rows):
+
+    lc = LatentCache(B, cap, swa_cap)
+    csa2_latent_append(lc, B, t, pos, latent, idx_k, swa)                 # any plane may be None
+    ws = LatentIndexWorkspace(B, 32, cap)
+    csa2_latent_index_topk(lc, B, 1, qpos, idx_q, 512, idx, ws, flags=CSA2_SCORE_RELU)   # 32 x 128 heads
+    csa2_latent_attend(lc, B, 1, qpos, q, idx, 512, out)                 # 64 heads x 512, tensor cores
 """
 from __future__ import annotations
 

@@ -337,7 +337,9 @@ CSA2_API csa2_status csa2_latent_append(const csa2_latent_cache* cache, int batc
  *   qpos [batch*tq] token of each row; idx [batch*tq][k] selected entries (-1 = none), each
  *   visible at its row ((qpos + 1) / ratio entries are); window tokens [max(swa_begin[b],
  *   qpos - win + 1, 0), qpos] with win <= 128 (swa_begin may be NULL: 0); sm_scale 0 gives
- *   1/sqrt(512); ratio 1 or 2 (the entry rule of csa2_shape.ratio).
+ *   1/sqrt(512); ratio 1 or 2 (the entry rule of csa2_shape.ratio). The window ring must hold
+ *   every window token of the call: with several rows per sequence, swa_cap >= win + the spread of
+ *   their positions.
  *   out [batch*tq][64][512] bf16; out_f32 (same shape, fp32) and lse [batch*tq][64] (natural
  *   log) may be NULL. A row with no key gives out = 0 and lse = -inf.
  *   ws: a workspace of at least 256 bytes initialised by csa2_workspace_init (its status word
