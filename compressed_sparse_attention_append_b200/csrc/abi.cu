@@ -288,7 +288,7 @@ const char* csa2_status_string(csa2_status s) {
     return "unknown status";
 }
 
-int csa2_version(void) { return 101; }
+int csa2_version(void) { return 200; }
 
 csa2_status csa2_workspace_size(const csa2_shape* shape, int batch, int tq, int k, int64_t max_scan, int pool_blocks,
                                 size_t* bytes) {

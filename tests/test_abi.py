@@ -84,11 +84,50 @@ int main(void) {
     assert out[7].strip() == csa.csa2_status_string(csa.CSA2_ERR_WORKSPACE)
 
 
+def test_plain_c_program_uses_the_latent_declarations(L):
+    """The latent cache struct and the entry points of the pages' own shapes, used from plain C:
+    MXFP4 entry bytes, the indexer's workspace size, and calls with an empty batch (no launch)."""
+    import subprocess
+    import tempfile
+
+    prog = r"""
+#include <stdio.h>
+#include <stdint.h>
+#include "csa2.h"
+int main(void) {
+    static uint8_t planes[5][4096] __attribute__((aligned(256)));
+    csa2_latent_cache c = {planes[0], planes[1], planes[2], planes[3], planes[4], 64, 128};
+    int64_t qpos[1] = {63};
+    uint16_t q[16] __attribute__((aligned(16))) = {0};
+    int32_t idx[1] = {-1};
+    size_t ws = 0;
+    int a = csa2_latent_index_workspace_size(2, 32, 64, &ws);
+    int b = csa2_latent_attend(&c, 0, 1, qpos, q, idx, 1, NULL, 128, 1, 0.f, q, NULL, NULL, NULL, 0, NULL);
+    int d = csa2_latent_append(&c, 0, 1, qpos, q, NULL, q, NULL, 0, NULL);
+    int e = csa2_latent_attend(&c, 1, 1, qpos, q, idx, 1, NULL, 200, 1, 0.f, q, NULL, NULL, NULL, 0, NULL);
+    printf("%zu %d %zu %d %d %d\n", csa2_mx_entry_bytes(128), a, ws, b, d, e);
+    return 0;
+}
+"""
+    libdir = os.path.dirname(csa.lib()._name)
+    with tempfile.TemporaryDirectory() as d:
+        c, exe = os.path.join(d, "p.c"), os.path.join(d, "p")
+        with open(c, "w") as f:
+            f.write(prog)
+        subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), c, "-o",
+                               exe, "-L", libdir, "-l:libcsa2.so", f"-Wl,-rpath,{libdir}"])
+        out = subprocess.run([exe], capture_output=True, text=True, timeout=60, check=True).stdout.split()
+    assert out[0] == "68" and out[1] == "0"
+    assert int(out[2]) == csa.csa2_latent_index_workspace_size(2, 32, 64)
+    assert out[3] == "0" and out[4] == "0"  # empty batches: nothing to do
+    assert int(out[5]) == csa.CSA2_ERR_UNSUPPORTED_SHAPE  # a window longer than 128
+
+
 def test_host_functions(L):
     assert csa.csa2_entry_bytes(256) == 144
     assert csa.csa2_entry_bytes(512) == 288
     assert csa.csa2_entry_bytes(24) == 0 and csa.csa2_entry_bytes(-16) == 0
-    assert csa.csa2_version() == 101
+    assert csa.csa2_version() == 200  # 0.2.0: the entry points of the pages' own shapes
     for s in range(7):
         assert csa.csa2_status_string(s)
     assert csa.csa2_status_string(99) == "unknown status"
