@@ -367,8 +367,9 @@ CSA2_API csa2_status csa2_latent_attend(const csa2_latent_cache* cache, int batc
  *   position order, padded with -1 (a row with qpos < 0 gives all -1).
  * Scores are evaluated exactly (integer block dots times power-of-two scales, fp64 sums) whenever
  * the 32-channel block maxima of a row's query and keys lie within 2^38 of each other.
- * ws: at least csa2_latent_index_workspace_size(batch*tq, hi, max_ctx) bytes, 256-byte aligned
- * (its first 4 bytes are the status word; the rest is scratch); max_ctx bounds the visible
+ * ws: at least csa2_latent_index_workspace_size(batch*tq, hi, max_ctx) bytes, 256-byte aligned and
+ * cleared once after allocation with csa2_workspace_init (its first 4 bytes are the status word,
+ * read and cleared by csa2_get_device_status; the rest is scratch); max_ctx bounds the visible
  * entries of every row: a row with more, or whose entries run past the capacity, sets
  * CSA2_DEV_BAD_POS and gives all -1. batch*tq <= 65535, 1 <= k <= 2048, ratio 1 or 2.
  */
